@@ -1,0 +1,404 @@
+"""CPU oracle for the MiniMax-H3 transformer block forward — TEST INFRASTRUCTURE.
+
+Only the tests, the package's ``smoke()`` check and the benchmark's CPU
+baseline may import this module. It is a plain, slow, float64 NumPy
+restatement of what the block computes, written to be checked against the
+pages by eye. It shares nothing with the CUDA path.
+
+Sources (titles and sections of the pages this follows):
+
+* [MX] "MiniMaxH3Transformer3DModel" (diffusers v0.43.0 docs): the overview
+  (one packed 1-D sequence, full self-attention, per-row modality tag selects
+  the AdaLN modulation; padding rows, tag -1, form their own attention
+  document under a boolean mask), the constructor parameters (56 heads of
+  128, hidden 5376, ffn 14336, freq_dim 256, time_embed_dim 2688 = input of
+  every AdaLN projection, rope_freq_dim 16 shared by the (t, h, w) axes with
+  2*3*16 channels rotated, rope_theta 1e4, norm_eps, qk_norm_eps) and the
+  ``forward`` arguments (timestep values, per-row timestep indices, tags,
+  positions, the three index tensors).
+* [ME] "MiniMax H3 Inference Engine voor Mac computers", sections
+  "Exacte DiT fusions" (gated attention residual followed by the MLP's AdaLN,
+  bf16 residual stream), "Checkpoint layout en media pipeline" (QKV rows
+  interleaved per attention head; fused QK-norm + RoPE), "Profiling en
+  diagnostische pads" (fc1 -> SwiGLU -> fc2).
+
+Readings where the pages leave a step open (each also listed in the design
+notes): LayerNorm without affine for the pre-norms; modulate as
+norm * (1 + scale) + shift with chunk order (shift1, scale1, gate1, shift2,
+scale2, gate2); per-row modulation = ada_table[tag] + tmod[t_idx] where
+tmod = W_proj . SiLU(TimeMLP(sinusoid(t))) is shared by all blocks; QK-norm is
+RMSNorm over a head's 128 channels with learned [128] weights; RoPE rotates
+channel pairs (32a + j, 32a + j + 16), a = t, h, w, with
+inv_freq[j] = theta^(-j/16); attention scale 1/sqrt(128); no biases; padding
+rows (tag -1) attend only padding rows and leave the block unchanged.
+
+Parity pins for every function here are in tests/test_oracle_pins.py.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Callable, Dict, Optional, Sequence, Tuple
+
+import numpy as np
+
+F = np.float64
+TAG_PAD = -1
+TILE = 128  # row-tile height used by the tile-class table of the layout step
+
+
+# --------------------------------------------------------------------------
+# Storage helpers
+# --------------------------------------------------------------------------
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of bf16 bit patterns (uint16) as float64."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(F)
+
+
+def round_bf16(a: np.ndarray) -> np.ndarray:
+    """Round to the nearest bf16 value (ties to even), through float32.
+
+    Used only by the optional bf16-storage emulation, which mimics a device
+    that holds fp32 values and stores them as bf16.
+    """
+    f = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << 16
+    return r.astype(np.uint32).view(np.float32).astype(F)
+
+
+def _store(a: np.ndarray, emulate: bool) -> np.ndarray:
+    return round_bf16(a) if emulate else a
+
+
+# --------------------------------------------------------------------------
+# a2: timestep embedding and the shared AdaLN projection  [MX: freq_dim,
+#     time_embed_hidden_dim, time_embed_dim; timesteps unscaled in [0, 1]]
+# --------------------------------------------------------------------------
+
+def silu(x: np.ndarray) -> np.ndarray:
+    return x / (1.0 + np.exp(-x))
+
+
+def timestep_sinusoid(t: np.ndarray, freq_dim: int) -> np.ndarray:
+    """[n_t] -> [n_t, freq_dim]: [cos(t f_i), sin(t f_i)], f_i = 10^4^(-i/(freq_dim/2))."""
+    half = freq_dim // 2
+    i = np.arange(half, dtype=F)
+    f = np.exp(-math.log(10000.0) * i / half)
+    arg = np.asarray(t, dtype=F)[:, None] * f[None, :]
+    return np.concatenate([np.cos(arg), np.sin(arg)], axis=1)
+
+
+def timestep_modulation(t: np.ndarray, w_t1: np.ndarray, w_t2: np.ndarray,
+                        w_proj: np.ndarray, freq_dim: int, hidden: int) -> np.ndarray:
+    """tmod[n_t, 6, H] = W_proj . SiLU(W_t2 . SiLU(W_t1 . sinusoid(t)))."""
+    s = timestep_sinusoid(t, freq_dim)
+    temb = silu(s @ np.asarray(w_t1, F).T) @ np.asarray(w_t2, F).T
+    tmod = silu(temb) @ np.asarray(w_proj, F).T
+    return tmod.reshape(-1, 6, hidden)
+
+
+# --------------------------------------------------------------------------
+# a3 / a7: norm + AdaLN modulate  [MX: norm_eps; per-row tag selects AdaLN]
+# --------------------------------------------------------------------------
+
+def row_modulation(tags: np.ndarray, t_idx: np.ndarray, ada_table: np.ndarray,
+                   tmod: np.ndarray) -> np.ndarray:
+    """[n] rows -> [n, 6, H]: ada_table[tag] + tmod[t_idx]; zero for padding rows."""
+    tags = np.asarray(tags)
+    table = np.asarray(ada_table, F)
+    m = np.zeros((tags.shape[0],) + table.shape[1:], F)
+    v = tags >= 0
+    m[v] = table[tags[v]] + np.asarray(tmod, F)[np.asarray(t_idx)[v]]
+    return m
+
+
+def layer_norm(x: np.ndarray, eps: float) -> np.ndarray:
+    """(x - mean) / sqrt(var + eps) over the last axis, biased variance, no affine."""
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps)
+
+
+def norm_modulate(x: np.ndarray, shift: np.ndarray, scale: np.ndarray,
+                  eps: float) -> np.ndarray:
+    return layer_norm(x, eps) * (1.0 + scale) + shift
+
+
+# --------------------------------------------------------------------------
+# a4: QKV projection, per-head QK-norm, 3-axis RoPE
+#     [MX: num_attention_heads * attention_head_dim > hidden_size;
+#      qk_norm_eps; rope_freq_dim, rope_theta]  [ME: QKV rows per head]
+# --------------------------------------------------------------------------
+
+def rms_norm(x: np.ndarray, w: np.ndarray, eps: float) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * w over the last axis."""
+    return x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps) * w
+
+
+def rope_inv_freq(rope_freq_dim: int, theta: float) -> np.ndarray:
+    j = np.arange(rope_freq_dim, dtype=F)
+    return theta ** (-j / rope_freq_dim)
+
+
+def rope_apply(x: np.ndarray, pos: np.ndarray, inv_freq: np.ndarray) -> np.ndarray:
+    """Rotate x[..., n, D] (n rows, any leading head axis after rows) by positions.
+
+    x has shape [n, NH, D]; pos [n, 3]. For axis a in (t, h, w) and j < nf,
+    the pair (c0, c1) = (2 nf a + j, 2 nf a + j + nf) is rotated by
+    angle pos[r, a] * inv_freq[j]. Channels >= 6 nf are left unchanged.
+    """
+    nf = inv_freq.shape[0]
+    out = np.array(x, dtype=F, copy=True)
+    for a in range(3):
+        ang = np.asarray(pos, F)[:, a:a + 1] * inv_freq[None, :]  # [n, nf]
+        c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+        lo = 2 * nf * a
+        x0 = x[:, :, lo:lo + nf]
+        x1 = x[:, :, lo + nf:lo + 2 * nf]
+        out[:, :, lo:lo + nf] = x0 * c - x1 * s
+        out[:, :, lo + nf:lo + 2 * nf] = x0 * s + x1 * c
+    return out
+
+
+def split_qkv_weight(w_qkv: np.ndarray, heads: int, head_dim: int) -> Tuple[np.ndarray, ...]:
+    """Head-interleaved [3 NH D, H] -> Wq, Wk, Wv each [NH D, H]."""
+    w = np.asarray(w_qkv).reshape(heads, 3, head_dim, -1)
+    return (w[:, 0].reshape(heads * head_dim, -1), w[:, 1].reshape(heads * head_dim, -1),
+            w[:, 2].reshape(heads * head_dim, -1))
+
+
+def split_w13(w13: np.ndarray, ffn: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Block-interleaved [2F, H] (128-row blocks W1_j, W3_j) -> W1, W3 each [F, H]."""
+    w = np.asarray(w13).reshape(ffn // 128, 2, 128, -1)
+    return w[:, 0].reshape(ffn, -1), w[:, 1].reshape(ffn, -1)
+
+
+def qkv_project(h: np.ndarray, pos: np.ndarray, w_qkv: np.ndarray, q_norm: np.ndarray,
+                k_norm: np.ndarray, dims, emulate: bool = False,
+                need_q: bool = True) -> Tuple[Optional[np.ndarray], np.ndarray, np.ndarray]:
+    """h [n, H] -> q, k, v [n, NH, D] after QK-norm and RoPE (q, k only)."""
+    NH, D = dims.heads, dims.head_dim
+    wq, wk, wv = split_qkv_weight(bf16_to_f64(w_qkv), NH, D)
+    inv = rope_inv_freq(dims.rope_freq_dim, dims.rope_theta)
+    qn, kn = bf16_to_f64(q_norm), bf16_to_f64(k_norm)
+    n = h.shape[0]
+    k = (h @ wk.T).reshape(n, NH, D)
+    v = (h @ wv.T).reshape(n, NH, D)
+    k = rope_apply(rms_norm(k, kn, dims.qk_norm_eps), pos, inv)
+    q = None
+    if need_q:
+        q = (h @ wq.T).reshape(n, NH, D)
+        q = _store(rope_apply(rms_norm(q, qn, dims.qk_norm_eps), pos, inv), emulate)
+    return q, _store(k, emulate), _store(v, emulate)
+
+
+# --------------------------------------------------------------------------
+# a5: bidirectional attention with the padding document
+#     [MX: padding rows stay in their own attention document]
+# --------------------------------------------------------------------------
+
+def attention(q: np.ndarray, doc_q: np.ndarray, k: np.ndarray, v: np.ndarray,
+              doc_k: np.ndarray, emulate: bool = False) -> np.ndarray:
+    """q [n, NH, D], k/v [S, NH, D]; keys visible where doc_k == doc_q.
+
+    Returns o [n, NH * D] = concat over heads of softmax(q k^T / sqrt(D)) v.
+    """
+    n, NH, D = q.shape
+    scale = 1.0 / math.sqrt(D)
+    o = np.empty((n, NH, D), F)
+    same = np.asarray(doc_q)[:, None] == np.asarray(doc_k)[None, :]
+    for hd in range(NH):
+        s = (q[:, hd, :] @ k[:, hd, :].T) * scale
+        s = np.where(same, s, -np.inf)
+        mx = s.max(axis=1, keepdims=True)
+        p = np.exp(s - mx)
+        l = p.sum(axis=1, keepdims=True)
+        p = _store(p, emulate)
+        o[:, hd, :] = (p @ v[:, hd, :]) / l
+    return _store(o.reshape(n, NH * D), emulate)
+
+
+# --------------------------------------------------------------------------
+# a6 .. a9: output projection, FFN, gated residuals  [ME: "Exacte DiT fusions"]
+# --------------------------------------------------------------------------
+
+def out_project_residual(x: np.ndarray, o: np.ndarray, gate: np.ndarray, w_o: np.ndarray,
+                         emulate: bool = False) -> np.ndarray:
+    """x1 = x + gate * (o W_o^T)."""
+    return _store(x + gate * (o @ bf16_to_f64(w_o).T), emulate)
+
+
+def ffn_gate(h2: np.ndarray, w13: np.ndarray, ffn: int, emulate: bool = False) -> np.ndarray:
+    """g = SiLU(h2 W1^T) * (h2 W3^T)."""
+    w1, w3 = split_w13(bf16_to_f64(w13), ffn)
+    return _store(silu(h2 @ w1.T) * (h2 @ w3.T), emulate)
+
+
+def ffn_down_residual(x1: np.ndarray, g: np.ndarray, gate: np.ndarray, w2: np.ndarray,
+                      emulate: bool = False) -> np.ndarray:
+    """x2 = x1 + gate * (g W2^T)."""
+    return _store(x1 + gate * (g @ bf16_to_f64(w2).T), emulate)
+
+
+# --------------------------------------------------------------------------
+# The block and the stack
+# --------------------------------------------------------------------------
+
+def _pre_attention(x, m, pos, w, dims, emulate, need_q=True):
+    h = _store(norm_modulate(x, m[:, 0], m[:, 1], dims.norm_eps), emulate)
+    return qkv_project(h, pos, w.w_qkv, w.q_norm, w.k_norm, dims, emulate, need_q)
+
+
+def _post_attention(x, o, m, w, dims, emulate):
+    x1 = out_project_residual(x, o, m[:, 2], w.w_o, emulate)
+    h2 = _store(norm_modulate(x1, m[:, 3], m[:, 4], dims.norm_eps), emulate)
+    g = ffn_gate(h2, w.w13, dims.ffn, emulate)
+    return ffn_down_residual(x1, g, m[:, 5], w.w2, emulate)
+
+
+def block_forward(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
+                  emulate: bool = False) -> np.ndarray:
+    """One block over the packed sequence. x [B, S, H] (values) -> [B, S, H] float64.
+
+    Padding rows (tag -1) are returned unchanged.
+    """
+    x = np.asarray(x, F)
+    tags = np.asarray(layout.tags)
+    if tags.shape[0] == 0:
+        return x.copy()
+    pad = tags < 0
+    m = row_modulation(tags, layout.t_idx, w.ada_table, tmod)
+    out = np.empty_like(x)
+    for b in range(x.shape[0]):
+        q, k, v = _pre_attention(x[b], m, layout.pos, w, dims, emulate)
+        o = attention(q, pad, k, v, pad, emulate)
+        y = _post_attention(x[b], o, m, w, dims, emulate)
+        out[b] = np.where(pad[:, None], x[b], y)
+    return out
+
+
+def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable[[np.ndarray], np.ndarray],
+                       dims, rows: np.ndarray, chunk: int = 2048) -> np.ndarray:
+    """The same block evaluated only at the query rows ``rows`` (B = 1).
+
+    Keys and values are needed for every row, so they are formed for all rows
+    in row chunks (each row's k and v depend on that row alone). ``tmod_rows``
+    maps timestep indices to their tmod rows [n, 6, H], so a caller with one
+    timestep per row never holds tmod for the whole sequence.
+    """
+    x = np.asarray(x, F)
+    S = x.shape[0]
+    tags = np.asarray(layout.tags)
+    pad = tags < 0
+    NH, D = dims.heads, dims.head_dim
+    K = np.empty((S, NH, D), F)
+    V = np.empty((S, NH, D), F)
+    table = np.asarray(w.ada_table, F)
+    for r0 in range(0, S, chunk):
+        r1 = min(S, r0 + chunk)
+        tg = tags[r0:r1]
+        m = np.zeros((r1 - r0, 6, dims.hidden), F)
+        vv = tg >= 0
+        if vv.any():
+            m[vv] = table[tg[vv]] + tmod_rows(np.asarray(layout.t_idx)[r0:r1][vv])
+        _, K[r0:r1], V[r0:r1] = _pre_attention(x[r0:r1], m, layout.pos[r0:r1], w, dims,
+                                               False, need_q=False)
+    rows = np.asarray(rows)
+    tg = tags[rows]
+    m = np.zeros((rows.shape[0], 6, dims.hidden), F)
+    vv = tg >= 0
+    if vv.any():
+        m[vv] = table[tg[vv]] + tmod_rows(np.asarray(layout.t_idx)[rows][vv])
+    q, _, _ = _pre_attention(x[rows], m, layout.pos[rows], w, dims, False)
+    o = attention(q, pad[rows], K, V, pad)
+    y = _post_attention(x[rows], o, m, w, dims, False)
+    return np.where(pad[rows][:, None], x[rows], y)
+
+
+def stack_forward(x: np.ndarray, weights_for_block: Callable[[int], object], n_blocks: int,
+                  layout, tmod: np.ndarray, dims, emulate: bool = False) -> np.ndarray:
+    """``n_blocks`` blocks in sequence, sharing one tmod (computed once per forward)."""
+    y = np.asarray(x, F)
+    for i in range(n_blocks):
+        y = block_forward(y, weights_for_block(i), layout, tmod, dims, emulate)
+    return y
+
+
+# --------------------------------------------------------------------------
+# a0 / a1: layout validation, tile classes, compaction, pack / unpack
+#          [MX: forward arguments; caller builds the packing]
+# --------------------------------------------------------------------------
+
+LAYOUT_OK = 0
+LAYOUT_BAD = -4
+
+
+def layout_check(layout, n_t: Optional[int] = None) -> int:
+    """0 if the layout is consistent, else -4.
+
+    Tags in {-1, 0, 1, 2}; every t_idx in [0, n_t); positions finite; each
+    index tensor in range, free of duplicates, pointing only at rows of its
+    modality, and as long as the number of such rows.
+    """
+    tags = np.asarray(layout.tags)
+    S = tags.shape[0]
+    nt = layout.timestep.shape[0] if n_t is None else n_t
+    if np.any((tags < -1) | (tags > 2)):
+        return LAYOUT_BAD
+    ti = np.asarray(layout.t_idx)
+    if ti.shape[0] != S or np.any((ti < 0) | (ti >= nt)):
+        return LAYOUT_BAD
+    if not np.all(np.isfinite(np.asarray(layout.pos))):
+        return LAYOUT_BAD
+    for idx, tag in ((layout.video_idx, 0), (layout.text_idx, 1), (layout.audio_idx, 2)):
+        idx = np.asarray(idx, np.int64)
+        if np.any((idx < 0) | (idx >= S)):
+            return LAYOUT_BAD
+        if np.unique(idx).shape[0] != idx.shape[0]:
+            return LAYOUT_BAD
+        if np.any(tags[idx] != tag):
+            return LAYOUT_BAD
+        if idx.shape[0] != int(np.count_nonzero(tags == tag)):
+            return LAYOUT_BAD
+    return LAYOUT_OK
+
+
+def tile_classes(tags: np.ndarray, tile: int = TILE) -> np.ndarray:
+    """Per row tile: 0 all rows valid, 1 all rows padding, 2 mixed."""
+    tags = np.asarray(tags)
+    S = tags.shape[0]
+    n = (S + tile - 1) // tile
+    out = np.zeros(n, np.uint8)
+    for i in range(n):
+        seg = tags[i * tile:min(S, (i + 1) * tile)]
+        npad = int(np.count_nonzero(seg < 0))
+        out[i] = 0 if npad == 0 else (1 if npad == seg.shape[0] else 2)
+    return out
+
+
+def compaction_perm(tags: np.ndarray) -> np.ndarray:
+    """Row order with valid rows first then padding rows, each in packed order."""
+    tags = np.asarray(tags)
+    return np.concatenate([np.nonzero(tags >= 0)[0], np.nonzero(tags < 0)[0]]).astype(np.int32)
+
+
+def pack_rows(layout, video: np.ndarray, audio: np.ndarray, text: np.ndarray,
+              H: int) -> np.ndarray:
+    """Scatter per-modality rows [B, N_m, H] into the packed [B, S, H]; padding rows 0."""
+    B = max(a.shape[0] for a in (video, audio, text))
+    out = np.zeros((B, layout.S, H), dtype=video.dtype)
+    for src, idx in ((video, layout.video_idx), (audio, layout.audio_idx),
+                     (text, layout.text_idx)):
+        for i, r in enumerate(np.asarray(idx)):
+            out[:, r] = src[:, i]
+    return out
+
+
+def unpack_rows(layout, x: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gather packed rows back to per-modality [B, N_m, H], in index order."""
+    return tuple(np.stack([x[:, r] for r in np.asarray(idx)], axis=1)
+                 if len(idx) else np.zeros((x.shape[0], 0, x.shape[2]), x.dtype)
+                 for idx in (layout.video_idx, layout.audio_idx, layout.text_idx))
