@@ -1,0 +1,469 @@
+// C ABI entry points: argument checks, layout object, block and stack
+// orchestration. Every step of the computation runs in this library's kernels.
+#include <stdio.h>
+
+#include <new>
+
+#include "internal.cuh"
+
+using namespace h3;
+
+namespace {
+
+inline cudaStream_t as_stream(h3_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+h3_status check_dims(const h3_dims* d) {
+  if (!d) return H3_ERR_ARG;
+  if (d->head_dim != 128 || d->rope_freq_dim != kRopeFreqs) return H3_ERR_SHAPE;
+  if (d->hidden <= 0 || d->hidden % 256 != 0 || d->hidden > 24 * 256) return H3_ERR_SHAPE;
+  if (d->heads <= 0 || d->heads % 2 != 0) return H3_ERR_SHAPE;
+  if (d->ffn <= 0 || d->ffn % 128 != 0) return H3_ERR_SHAPE;
+  if (d->n_modalities < 3) return H3_ERR_SHAPE;
+  if (d->freq_dim <= 0 || d->freq_dim % 2 != 0 || d->time_hidden <= 0 || d->time_embed_dim <= 0)
+    return H3_ERR_SHAPE;
+  if (!(d->norm_eps > 0.f) || !(d->qk_norm_eps > 0.f) || !(d->rope_theta > 0.f))
+    return H3_ERR_ARG;
+  return H3_OK;
+}
+
+inline h3_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return H3_OK;
+  if (e == cudaErrorInvalidValue) return H3_ERR_ARG;
+  return H3_ERR_CUDA;
+}
+
+#define H3_TRY(expr)                      \
+  do {                                    \
+    const h3_status _s = (expr);          \
+    if (_s != H3_OK) return _s;           \
+  } while (0)
+
+#define H3_CUDA(expr) H3_TRY(cuda_status(expr))
+
+struct Workspace {
+  void *h, *qkv_g, *o, *xc;
+  void *q, *k, *v, *g;
+};
+
+size_t ws_parts(const h3_dims& d, int B, int S, Workspace* w, void* base) {
+  const size_t rows = (size_t)B * S;
+  const size_t A = (size_t)d.heads * d.head_dim;
+  const size_t h_b = align256(rows * d.hidden * 2);
+  const size_t one_b = align256(rows * A * 2);          // q, k, v each
+  const size_t g_b = align256(rows * (size_t)d.ffn * 2);  // g reuses the q/k/v region
+  const size_t qg_b = 3 * one_b > g_b ? 3 * one_b : g_b;
+  const size_t o_b = align256(rows * A * 2);
+  const size_t xc_b = align256(rows * d.hidden * 2);
+  if (w) {
+    uint8_t* p = static_cast<uint8_t*>(base);
+    w->h = p;
+    w->qkv_g = p + h_b;
+    w->o = p + h_b + qg_b;
+    w->xc = p + h_b + qg_b + o_b;
+    w->q = w->qkv_g;
+    w->k = static_cast<uint8_t*>(w->qkv_g) + one_b;
+    w->v = static_cast<uint8_t*>(w->qkv_g) + 2 * one_b;
+    w->g = w->qkv_g;
+  }
+  return h_b + qg_b + o_b + xc_b;
+}
+
+h3_status check_weights(const h3_block_weights* w) {
+  if (!w || !w->w_qkv || !w->q_norm || !w->k_norm || !w->w_o || !w->w13 || !w->w2 ||
+      !w->ada_table)
+    return H3_ERR_ARG;
+  if (!aligned16(w->w_qkv) || !aligned16(w->q_norm) || !aligned16(w->k_norm) ||
+      !aligned16(w->w_o) || !aligned16(w->w13) || !aligned16(w->w2) || !aligned16(w->ada_table))
+    return H3_ERR_ALIGN;
+  return H3_OK;
+}
+
+// One block over the rows described by `L` (full or compacted view), in place on x.
+h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutView& L,
+                    const float* tmod, void* x, int B, const Workspace& ws, cudaStream_t st) {
+  const int M = B * L.S;
+  if (M == 0) return H3_OK;
+  const int H = d.hidden, A = d.heads * d.head_dim, Fd = d.ffn;
+  H3_CUDA(launch_norm_modulate(L, B, H, 0, 1, d.norm_eps, x, w.ada_table, tmod, ws.h, st));
+  GemmEpiArgs e;
+  e.L = L;
+  e.B = B;
+  e.NH = d.heads;
+  e.q = ws.q;
+  e.k = ws.k;
+  e.v = ws.v;
+  e.q_norm = w.q_norm;
+  e.k_norm = w.k_norm;
+  e.qk_eps = d.qk_norm_eps;
+  H3_CUDA(launch_gemm(EPI_QKV, M, 3 * A, H, ws.h, w.w_qkv, e, st));
+  H3_CUDA(launch_attention(L, B, d.heads, ws.q, ws.k, ws.v, ws.o, st));
+  GemmEpiArgs r;
+  r.L = L;
+  r.B = B;
+  r.x = x;
+  r.table = w.ada_table;
+  r.tmod = tmod;
+  r.gate_chunk = 2;
+  H3_CUDA(launch_gemm(EPI_RESID, M, H, A, ws.o, w.w_o, r, st));
+  H3_CUDA(launch_norm_modulate(L, B, H, 3, 4, d.norm_eps, x, w.ada_table, tmod, ws.h, st));
+  GemmEpiArgs sg;
+  sg.L = L;
+  sg.out = ws.g;
+  H3_CUDA(launch_gemm(EPI_SWIGLU, M, 2 * Fd, H, ws.h, w.w13, sg, st));
+  r.gate_chunk = 5;
+  H3_CUDA(launch_gemm(EPI_RESID, M, H, Fd, ws.g, w.w2, r, st));
+  return H3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* h3_status_string(h3_status s) {
+  switch (s) {
+    case H3_OK: return "ok";
+    case H3_ERR_ARG: return "invalid argument";
+    case H3_ERR_SHAPE: return "unsupported shape";
+    case H3_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case H3_ERR_LAYOUT: return "inconsistent packed layout";
+    case H3_ERR_WORKSPACE: return "workspace too small";
+    case H3_ERR_CUDA: return "CUDA error";
+    case H3_ERR_TIMEOUT: return "bounded in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+int h3_abi_version(void) { return 1; }
+
+h3_status h3_layout_prepare(const h3_dims* dims, const h3_layout_desc* desc, h3_stream_t stream,
+                            h3_layout_t* out) {
+  if (!out || !desc) return H3_ERR_ARG;
+  *out = nullptr;
+  H3_TRY(check_dims(dims));
+  const int S = desc->S;
+  if (S < 0 || desc->n_t < 0 || desc->n_video < 0 || desc->n_audio < 0 || desc->n_text < 0)
+    return H3_ERR_ARG;
+  if (S > 0 && (!desc->pos || !desc->tags || !desc->t_idx)) return H3_ERR_ARG;
+  if ((desc->n_video && !desc->video_idx) || (desc->n_audio && !desc->audio_idx) ||
+      (desc->n_text && !desc->text_idx))
+    return H3_ERR_ARG;
+  if (desc->n_video + desc->n_audio + desc->n_text > S) return H3_ERR_LAYOUT;
+  cudaStream_t st = as_stream(stream);
+  h3_layout* L = new (std::nothrow) h3_layout();
+  if (!L) return H3_ERR_CUDA;
+  cudaGetDevice(&L->device);
+  L->S = S;
+  L->n_t = desc->n_t;
+  L->n_video = desc->n_video;
+  L->n_audio = desc->n_audio;
+  L->n_text = desc->n_text;
+  L->n_tiles = (S + kTile - 1) / kTile;
+  const size_t nt = L->n_tiles;
+  const size_t sz_i = align256((size_t)S * 4), sz_pos = align256((size_t)S * 12),
+               sz_rope = align256((size_t)S * kRopePairs * 8), sz_tc = align256(nt),
+               sz_kv = align256(nt * 16);
+  const size_t total = 6 * sz_i /*tags t_idx src perm c_tags c_tidx*/ + sz_pos + 2 * sz_rope +
+                       2 * sz_tc + 2 * sz_kv + align256((size_t)desc->n_video * 4) +
+                       align256((size_t)desc->n_audio * 4) + align256((size_t)desc->n_text * 4) +
+                       256 /*err*/;
+  if (cudaMalloc(&L->block, total) != cudaSuccess) {
+    delete L;
+    return H3_ERR_CUDA;
+  }
+  uint8_t* p = static_cast<uint8_t*>(L->block);
+  auto take = [&](size_t n) {
+    uint8_t* q = p;
+    p += n;
+    return q;
+  };
+  L->tags = reinterpret_cast<int32_t*>(take(sz_i));
+  L->t_idx = reinterpret_cast<int32_t*>(take(sz_i));
+  L->src_of_row = reinterpret_cast<int32_t*>(take(sz_i));
+  L->perm = reinterpret_cast<int32_t*>(take(sz_i));
+  L->c_tags = reinterpret_cast<int32_t*>(take(sz_i));
+  L->c_tidx = reinterpret_cast<int32_t*>(take(sz_i));
+  L->pos = reinterpret_cast<float*>(take(sz_pos));
+  L->rope = reinterpret_cast<float2*>(take(sz_rope));
+  L->c_rope = reinterpret_cast<float2*>(take(sz_rope));
+  L->tile_class = take(sz_tc);
+  L->c_tile_class = take(sz_tc);
+  L->key_valid = reinterpret_cast<uint32_t*>(take(sz_kv));
+  L->c_key_valid = reinterpret_cast<uint32_t*>(take(sz_kv));
+  L->video_idx = reinterpret_cast<int32_t*>(take(align256((size_t)desc->n_video * 4)));
+  L->audio_idx = reinterpret_cast<int32_t*>(take(align256((size_t)desc->n_audio * 4)));
+  L->text_idx = reinterpret_cast<int32_t*>(take(align256((size_t)desc->n_text * 4)));
+  L->err = reinterpret_cast<int*>(take(256));
+
+  h3_status rc = H3_OK;
+  int32_t* scratch = nullptr;  // hits[S], tile_pad[n_tiles], counts[4], n_valid, status
+  const size_t scratch_n = (size_t)S + nt + 4 + 1 + 1;
+  int host_st[2] = {0, 0};
+  do {
+    if (cudaMalloc(&scratch, scratch_n * 4) != cudaSuccess) { rc = H3_ERR_CUDA; break; }
+    if (cudaMemsetAsync(scratch, 0, scratch_n * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(L->err, 0, 256, st) != cudaSuccess) { rc = H3_ERR_CUDA; break; }
+    bool cp_ok = true;
+    if (S > 0) {
+      cp_ok &= cudaMemcpyAsync(L->tags, desc->tags, (size_t)S * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+      cp_ok &= cudaMemcpyAsync(L->t_idx, desc->t_idx, (size_t)S * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+      cp_ok &= cudaMemcpyAsync(L->pos, desc->pos, (size_t)S * 12, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    }
+    if (desc->n_video)
+      cp_ok &= cudaMemcpyAsync(L->video_idx, desc->video_idx, (size_t)desc->n_video * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    if (desc->n_audio)
+      cp_ok &= cudaMemcpyAsync(L->audio_idx, desc->audio_idx, (size_t)desc->n_audio * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    if (desc->n_text)
+      cp_ok &= cudaMemcpyAsync(L->text_idx, desc->text_idx, (size_t)desc->n_text * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    if (!cp_ok) { rc = H3_ERR_CUDA; break; }
+    int* d_status = scratch + S + nt + 5;
+    if (launch_layout_prepare(L, dims->rope_theta, d_status, scratch, st) != cudaSuccess) {
+      rc = H3_ERR_CUDA;
+      break;
+    }
+    // n_valid (scratch[S + nt + 4]) and status are adjacent
+    if (cudaMemcpyAsync(host_st, scratch + S + nt + 4, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+      rc = H3_ERR_CUDA;
+      break;
+    }
+    if (host_st[1] != 0) { rc = H3_ERR_LAYOUT; break; }
+    L->n_valid = host_st[0];
+    L->c_tiles = (L->n_valid + kTile - 1) / kTile;
+    if (launch_compact_tables(L, st) != cudaSuccess) { rc = H3_ERR_CUDA; break; }
+    L->tile_class_host.resize(nt);
+    if (nt && cudaMemcpyAsync(L->tile_class_host.data(), L->tile_class, nt, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+      rc = H3_ERR_CUDA;
+      break;
+    }
+    if (cudaStreamSynchronize(st) != cudaSuccess) { rc = H3_ERR_CUDA; break; }
+  } while (0);
+  if (scratch) cudaFree(scratch);
+  if (rc != H3_OK) {
+    cudaFree(L->block);
+    delete L;
+    return rc;
+  }
+  *out = L;
+  return H3_OK;
+}
+
+void h3_layout_destroy(h3_layout_t L) {
+  if (!L) return;
+  cudaDeviceSynchronize();
+  cudaFree(L->block);
+  delete L;
+}
+
+h3_status h3_layout_error(h3_layout_t L) {
+  if (!L) return H3_ERR_ARG;
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return H3_ERR_CUDA;
+  if (cudaMemcpy(&v, L->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return H3_ERR_CUDA;
+  if (v != 0 && cudaMemset(L->err, 0, 4) != cudaSuccess) return H3_ERR_CUDA;
+  return v == 0 ? H3_OK : H3_ERR_TIMEOUT;
+}
+
+h3_status h3_layout_export(h3_layout_t L, int32_t* perm_host, uint8_t* tile_class_host,
+                           int32_t* n_valid_host) {
+  if (!L) return H3_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return H3_ERR_CUDA;
+  if (perm_host && L->S > 0 &&
+      cudaMemcpy(perm_host, L->perm, (size_t)L->S * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return H3_ERR_CUDA;
+  if (tile_class_host && L->n_tiles > 0 &&
+      cudaMemcpy(tile_class_host, L->tile_class, L->n_tiles, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return H3_ERR_CUDA;
+  if (n_valid_host) *n_valid_host = L->n_valid;
+  return H3_OK;
+}
+
+size_t h3_workspace_size(const h3_dims* dims, int B, int S) {
+  if (check_dims(dims) != H3_OK || B < 0 || S < 0) return 0;
+  return ws_parts(*dims, B, S, nullptr, nullptr);
+}
+
+h3_status h3_pack_rows(h3_layout_t L, int B, int row_elems, const void* video, const void* audio,
+                       const void* text, void* x_packed, h3_stream_t stream) {
+  if (!L || B < 0 || row_elems <= 0 || !x_packed) return H3_ERR_ARG;
+  if (row_elems % 8 != 0) return H3_ERR_SHAPE;
+  if ((L->n_video && !video) || (L->n_audio && !audio) || (L->n_text && !text)) return H3_ERR_ARG;
+  if (!aligned16(video) || !aligned16(audio) || !aligned16(text) || !aligned16(x_packed))
+    return H3_ERR_ALIGN;
+  H3_CUDA(launch_pack(L, B, row_elems, video, audio, text, x_packed, as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_unpack_rows(h3_layout_t L, int B, int row_elems, const void* x_packed, void* video,
+                         void* audio, void* text, h3_stream_t stream) {
+  if (!L || B < 0 || row_elems <= 0 || !x_packed) return H3_ERR_ARG;
+  if (row_elems % 8 != 0) return H3_ERR_SHAPE;
+  if (!aligned16(video) || !aligned16(audio) || !aligned16(text) || !aligned16(x_packed))
+    return H3_ERR_ALIGN;
+  H3_CUDA(launch_unpack(L, B, row_elems, x_packed, video, audio, text, as_stream(stream)));
+  return H3_OK;
+}
+
+size_t h3_timestep_workspace_size(const h3_dims* dims, int n_t) {
+  if (check_dims(dims) != H3_OK || n_t < 0) return 0;
+  return align256((size_t)n_t * (dims->freq_dim + dims->time_hidden + dims->time_embed_dim) * 4);
+}
+
+h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const float* t, const float* w_t1,
+                                 const float* w_t2, const float* w_proj, float* tmod, void* ws,
+                                 size_t ws_bytes, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (n_t < 0) return H3_ERR_ARG;
+  if (n_t == 0) return H3_OK;
+  if (!t || !w_t1 || !w_t2 || !w_proj || !tmod || !ws) return H3_ERR_ARG;
+  if (!aligned16(t) || !aligned16(w_t1) || !aligned16(w_t2) || !aligned16(w_proj) ||
+      !aligned16(tmod) || !aligned16(ws))
+    return H3_ERR_ALIGN;
+  if (ws_bytes < h3_timestep_workspace_size(dims, n_t)) return H3_ERR_WORKSPACE;
+  H3_CUDA(launch_timestep(*dims, n_t, t, w_t1, w_t2, w_proj, tmod, static_cast<float*>(ws),
+                          as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_norm_modulate(const h3_dims* dims, h3_layout_t L, int B, int which, const void* x,
+                           const float* ada_table, const float* tmod, void* h,
+                           h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || (which != 0 && which != 1) || !x || !ada_table || !tmod || !h)
+    return H3_ERR_ARG;
+  if (!aligned16(x) || !aligned16(ada_table) || !aligned16(tmod) || !aligned16(h))
+    return H3_ERR_ALIGN;
+  const int c0 = which == 0 ? 0 : 3;
+  H3_CUDA(launch_norm_modulate(L->view(), B, dims->hidden, c0, c0 + 1, dims->norm_eps, x,
+                               ada_table, tmod, h, as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_qkv_rope(const h3_dims* dims, h3_layout_t L, int B, const void* h, const void* w_qkv,
+                      const void* q_norm, const void* k_norm, void* q, void* k, void* v,
+                      h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !h || !w_qkv || !q_norm || !k_norm || !q || !k || !v) return H3_ERR_ARG;
+  if (!aligned16(h) || !aligned16(w_qkv) || !aligned16(q_norm) || !aligned16(k_norm) ||
+      !aligned16(q) || !aligned16(k) || !aligned16(v))
+    return H3_ERR_ALIGN;
+  GemmEpiArgs e;
+  e.L = L->view();
+  e.B = B;
+  e.NH = dims->heads;
+  e.q = q;
+  e.k = k;
+  e.v = v;
+  e.q_norm = q_norm;
+  e.k_norm = k_norm;
+  e.qk_eps = dims->qk_norm_eps;
+  H3_CUDA(launch_gemm(EPI_QKV, B * L->S, 3 * dims->heads * dims->head_dim, dims->hidden, h,
+                      w_qkv, e, as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_attention(const h3_dims* dims, h3_layout_t L, int B, const void* q, const void* k,
+                       const void* v, void* o, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !q || !k || !v || !o) return H3_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return H3_ERR_ALIGN;
+  H3_CUDA(launch_attention(L->view(), B, dims->heads, q, k, v, o, as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_out_residual(const h3_dims* dims, h3_layout_t L, int B, const void* o,
+                          const void* w_o, const float* ada_table, const float* tmod, void* x,
+                          h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !o || !w_o || !ada_table || !tmod || !x) return H3_ERR_ARG;
+  if (!aligned16(o) || !aligned16(w_o) || !aligned16(ada_table) || !aligned16(tmod) ||
+      !aligned16(x))
+    return H3_ERR_ALIGN;
+  GemmEpiArgs r;
+  r.L = L->view();
+  r.B = B;
+  r.x = x;
+  r.table = ada_table;
+  r.tmod = tmod;
+  r.gate_chunk = 2;
+  H3_CUDA(launch_gemm(EPI_RESID, B * L->S, dims->hidden, dims->heads * dims->head_dim, o, w_o, r,
+                      as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_ffn_up(const h3_dims* dims, h3_layout_t L, int B, const void* h2, const void* w13,
+                    void* g, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !h2 || !w13 || !g) return H3_ERR_ARG;
+  if (!aligned16(h2) || !aligned16(w13) || !aligned16(g)) return H3_ERR_ALIGN;
+  GemmEpiArgs sg;
+  sg.L = L->view();
+  sg.out = g;
+  H3_CUDA(launch_gemm(EPI_SWIGLU, B * L->S, 2 * dims->ffn, dims->hidden, h2, w13, sg,
+                      as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_ffn_down_residual(const h3_dims* dims, h3_layout_t L, int B, const void* g,
+                               const void* w2, const float* ada_table, const float* tmod,
+                               void* x, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !g || !w2 || !ada_table || !tmod || !x) return H3_ERR_ARG;
+  if (!aligned16(g) || !aligned16(w2) || !aligned16(ada_table) || !aligned16(tmod) ||
+      !aligned16(x))
+    return H3_ERR_ALIGN;
+  GemmEpiArgs r;
+  r.L = L->view();
+  r.B = B;
+  r.x = x;
+  r.table = ada_table;
+  r.tmod = tmod;
+  r.gate_chunk = 5;
+  H3_CUDA(launch_gemm(EPI_RESID, B * L->S, dims->hidden, dims->ffn, g, w2, r, as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_block_forward(const h3_dims* dims, const h3_block_weights* weights, h3_layout_t L,
+                           const float* tmod, void* x, int B, void* ws, size_t ws_bytes,
+                           h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !tmod || !x || !ws) return H3_ERR_ARG;
+  H3_TRY(check_weights(weights));
+  if (!aligned16(tmod) || !aligned16(x) || !aligned16(ws)) return H3_ERR_ALIGN;
+  if (ws_bytes < h3_workspace_size(dims, B, L->S)) return H3_ERR_WORKSPACE;
+  Workspace w;
+  ws_parts(*dims, B, L->S, &w, ws);
+  return run_block(*dims, *weights, L->view(), tmod, x, B, w, as_stream(stream));
+}
+
+h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* weights, int n_blocks,
+                           h3_layout_t L, const float* tmod, void* x, int B, void* ws,
+                           size_t ws_bytes, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || n_blocks < 0 || !tmod || !x || !ws || (n_blocks > 0 && !weights))
+    return H3_ERR_ARG;
+  for (int i = 0; i < n_blocks; ++i) H3_TRY(check_weights(&weights[i]));
+  if (!aligned16(tmod) || !aligned16(x) || !aligned16(ws)) return H3_ERR_ALIGN;
+  if (ws_bytes < h3_workspace_size(dims, B, L->S)) return H3_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  Workspace w;
+  ws_parts(*dims, B, L->S, &w, ws);
+  if (L->n_valid == L->S) {
+    for (int i = 0; i < n_blocks; ++i)
+      H3_TRY(run_block(*dims, weights[i], L->view(), tmod, x, B, w, st));
+    return H3_OK;
+  }
+  // Valid rows never see padding rows, and padding rows leave every block
+  // unchanged, so the blocks run on the compacted valid rows alone.
+  const int V = L->n_valid;
+  H3_CUDA(launch_permute_rows(B, V, L->S, dims->hidden, L->perm, x, w.xc, true, st));
+  for (int i = 0; i < n_blocks; ++i)
+    H3_TRY(run_block(*dims, weights[i], L->compact_view(), tmod, w.xc, B, w, st));
+  H3_CUDA(launch_permute_rows(B, V, L->S, dims->hidden, L->perm, w.xc, x, false, st));
+  return H3_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/h3.h"
+
+namespace h3 {
+
+constexpr int kTile = 128;        // row tile (attention q/kv tiles, GEMM M tile)
+constexpr int kRopeFreqs = 16;    // rope_freq_dim supported by the kernels
+constexpr int kRopePairs = 3 * kRopeFreqs;  // (cos, sin) entries per row
+
+// Device view of a packed layout, passed by value to kernels.
+struct LayoutView {
+  int S;                    // rows per batch element
+  int n_tiles;              // ceil(S / 128)
+  const int32_t* tags;      // [S]
+  const int32_t* t_idx;     // [S]
+  const float2* rope;       // [S, 48] (cos, sin) of pos[r][a] * inv_freq[j], index 16a + j
+  const uint8_t* tile_class;  // [n_tiles] 0 valid, 1 padding, 2 mixed
+  const uint32_t* key_valid;  // [n_tiles * 4] bit i of word w: row 128 t + 32 w + i is valid
+  int* err;                 // device error word
+};
+
+}  // namespace h3
+
+// The opaque layout object of the C ABI.
+struct h3_layout {
+  int S = 0, n_t = 0, n_video = 0, n_audio = 0, n_text = 0, n_valid = 0, n_tiles = 0;
+  int device = 0;
+  void* block = nullptr;  // single device allocation holding every table
+  int32_t *tags = nullptr, *t_idx = nullptr, *video_idx = nullptr, *audio_idx = nullptr,
+          *text_idx = nullptr, *src_of_row = nullptr, *perm = nullptr;
+  float* pos = nullptr;
+  float2* rope = nullptr;
+  uint8_t* tile_class = nullptr;
+  uint32_t* key_valid = nullptr;
+  // compacted (valid rows only) view
+  int32_t *c_tags = nullptr, *c_tidx = nullptr;
+  float2* c_rope = nullptr;
+  uint8_t* c_tile_class = nullptr;
+  uint32_t* c_key_valid = nullptr;
+  int c_tiles = 0;
+  int* err = nullptr;
+  std::vector<uint8_t> tile_class_host;
+
+  h3::LayoutView view() const {
+    return h3::LayoutView{S, n_tiles, tags, t_idx, rope, tile_class, key_valid, err};
+  }
+  h3::LayoutView compact_view() const {
+    return h3::LayoutView{n_valid, c_tiles, c_tags, c_tidx, c_rope, c_tile_class, c_key_valid,
+                          err};
+  }
+};
+
+namespace h3 {
+
+// ---- launchers (each returns cudaError_t of the launch) ----
+
+cudaError_t launch_layout_prepare(h3_layout* L, float rope_theta, int* d_status,
+                                  int32_t* d_scratch, cudaStream_t st);
+cudaError_t launch_compact_tables(h3_layout* L, cudaStream_t st);
+cudaError_t launch_pack(const h3_layout* L, int B, int row_elems, const void* video,
+                        const void* audio, const void* text, void* x, cudaStream_t st);
+cudaError_t launch_unpack(const h3_layout* L, int B, int row_elems, const void* x, void* video,
+                          void* audio, void* text, cudaStream_t st);
+// dst[b, j] = src[b, perm[j]] (gather == true, src [B, S_src, E], dst [B, n, E])
+// dst[b, perm[j]] = src[b, j] (gather == false, src [B, n, E], dst [B, S_dst, E])
+cudaError_t launch_permute_rows(int B, int n, int S_full, int row_elems, const int32_t* perm,
+                                const void* src, void* dst, bool gather, cudaStream_t st);
+
+cudaError_t launch_norm_modulate(const LayoutView& L, int B, int H, int chunk_shift,
+                                 int chunk_scale, float eps, const void* x, const float* table,
+                                 const float* tmod, void* h, cudaStream_t st);
+
+cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const float* w_t1,
+                            const float* w_t2, const float* w_proj, float* tmod, float* ws,
+                            cudaStream_t st);
+
+enum GemmEpilogue { EPI_STORE = 0, EPI_QKV = 1, EPI_RESID = 2, EPI_SWIGLU = 3 };
+
+struct GemmEpiArgs {
+  LayoutView L;
+  int B = 1, NH = 0;
+  // EPI_STORE: out [M, N]; EPI_SWIGLU: out [M, N/2]
+  void* out = nullptr;
+  // EPI_QKV
+  void *q = nullptr, *k = nullptr, *v = nullptr;
+  const void *q_norm = nullptr, *k_norm = nullptr;
+  float qk_eps = 0.f;
+  // EPI_RESID: x [M, N] in/out, gate = table[tag][gate_chunk] + tmod[t_idx][gate_chunk]
+  void* x = nullptr;
+  const float* table = nullptr;
+  const float* tmod = nullptr;
+  int gate_chunk = 0;
+};
+
+// C[M, N] epilogue( A[M, K] . B[N, K]^T ), bf16 in, fp32 accumulate.
+cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void* Bm,
+                        const GemmEpiArgs& e, cudaStream_t st);
+
+cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, const void* k,
+                             const void* v, void* o, cudaStream_t st);
+
+int num_sms();
+
+}  // namespace h3

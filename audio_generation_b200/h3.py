@@ -1,0 +1,288 @@
+"""ctypes binding of the C ABI in include/h3.h (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+computation of its own: it turns tensors into device pointers, checks the
+returned status and raises ``H3Error`` on failure. Device memory, streams and
+tensors come from PyTorch; all of the block's arithmetic runs in libh3.so.
+
+The library must be built (``python -m audio_generation_b200.build``); there is
+no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libh3.so")
+
+H3_OK = 0
+H3_ERR_ARG = -1
+H3_ERR_SHAPE = -2
+H3_ERR_ALIGN = -3
+H3_ERR_LAYOUT = -4
+H3_ERR_WORKSPACE = -5
+H3_ERR_CUDA = -6
+H3_ERR_TIMEOUT = -7
+
+
+class H3Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {h3_status_string(status)} ({status})")
+
+
+class h3_dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "hidden", "heads", "head_dim", "ffn", "time_embed_dim", "time_hidden", "freq_dim",
+        "rope_freq_dim", "n_modalities")] + [
+        ("rope_theta", ctypes.c_float), ("norm_eps", ctypes.c_float),
+        ("qk_norm_eps", ctypes.c_float)]
+
+
+class h3_layout_desc(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_int), ("n_t", ctypes.c_int), ("n_video", ctypes.c_int),
+                ("n_audio", ctypes.c_int), ("n_text", ctypes.c_int),
+                ("pos", ctypes.c_void_p), ("tags", ctypes.c_void_p), ("t_idx", ctypes.c_void_p),
+                ("video_idx", ctypes.c_void_p), ("audio_idx", ctypes.c_void_p),
+                ("text_idx", ctypes.c_void_p)]
+
+
+class h3_block_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_qkv", "q_norm", "k_norm", "w_o", "w13", "w2", "ada_table")]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_SIGNATURES = {
+    "h3_status_string": (ctypes.c_char_p, [_i]),
+    "h3_abi_version": (_i, []),
+    "h3_layout_prepare": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_layout_desc), _vp,
+                               ctypes.POINTER(_vp)]),
+    "h3_layout_destroy": (None, [_vp]),
+    "h3_layout_error": (_i, [_vp]),
+    "h3_layout_export": (_i, [_vp, _vp, _vp, _vp]),
+    "h3_workspace_size": (_sz, [ctypes.POINTER(h3_dims), _i, _i]),
+    "h3_pack_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "h3_unpack_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "h3_timestep_workspace_size": (_sz, [ctypes.POINTER(h3_dims), _i]),
+    "h3_timestep_modulation": (_i, [ctypes.POINTER(h3_dims), _i, _vp, _vp, _vp, _vp, _vp, _vp,
+                                    _sz, _vp]),
+    "h3_norm_modulate": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "h3_qkv_rope": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                         _vp]),
+    "h3_attention": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp]),
+    "h3_out_residual": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "h3_ffn_up": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp]),
+    "h3_ffn_down_residual": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp,
+                                  _vp]),
+    "h3_block_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _vp,
+                              _vp, _vp, _i, _vp, _sz, _vp]),
+    "h3_stack_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _i, _vp,
+                              _vp, _vp, _i, _vp, _sz, _vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libh3.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m audio_generation_b200.build` (no fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- marshalling helpers
+
+def _ptr(t) -> Optional[int]:
+    """Device (or host) address of a tensor / int / None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != H3_OK:
+        raise H3Error(status, where)
+
+
+def make_dims(d) -> h3_dims:
+    """h3_dims from any object with the constructor-parameter attributes."""
+    return h3_dims(hidden=d.hidden, heads=d.heads, head_dim=d.head_dim, ffn=d.ffn,
+                   time_embed_dim=d.time_embed_dim, time_hidden=d.time_hidden,
+                   freq_dim=d.freq_dim, rope_freq_dim=d.rope_freq_dim,
+                   n_modalities=getattr(d, "n_modalities", 3), rope_theta=d.rope_theta,
+                   norm_eps=d.norm_eps, qk_norm_eps=d.qk_norm_eps)
+
+
+def make_block_weights(w_qkv, q_norm, k_norm, w_o, w13, w2, ada_table) -> h3_block_weights:
+    return h3_block_weights(*[_ptr(t) for t in (w_qkv, q_norm, k_norm, w_o, w13, w2, ada_table)])
+
+
+# ---------------------------------------------------------------- entry points
+
+def h3_status_string(status: int) -> str:
+    return lib().h3_status_string(status).decode()
+
+
+def h3_abi_version() -> int:
+    return lib().h3_abi_version()
+
+
+class Layout:
+    """Owns an h3_layout_t; released by close() or garbage collection."""
+
+    def __init__(self, handle: int, S: int):
+        self.handle = handle
+        self.S = S
+
+    def close(self) -> None:
+        if self.handle:
+            lib().h3_layout_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def _as_param_(self):
+        return self.handle
+
+
+def h3_layout_prepare(dims: h3_dims, S: int, n_t: int, pos, tags, t_idx, video_idx, audio_idx,
+                      text_idx, stream=None) -> Layout:
+    desc = h3_layout_desc(S=S, n_t=n_t, n_video=_numel(video_idx), n_audio=_numel(audio_idx),
+                          n_text=_numel(text_idx), pos=_ptr(pos), tags=_ptr(tags),
+                          t_idx=_ptr(t_idx), video_idx=_ptr(video_idx),
+                          audio_idx=_ptr(audio_idx), text_idx=_ptr(text_idx))
+    out = ctypes.c_void_p()
+    _check(lib().h3_layout_prepare(ctypes.byref(dims), ctypes.byref(desc), _stream(stream),
+                                   ctypes.byref(out)), "h3_layout_prepare")
+    return Layout(out.value, S)
+
+
+def _numel(t) -> int:
+    return 0 if t is None else int(t.numel())
+
+
+def h3_layout_destroy(layout: Layout) -> None:
+    layout.close()
+
+
+def h3_layout_error(layout: Layout) -> int:
+    return lib().h3_layout_error(layout.handle)
+
+
+def h3_layout_export(layout: Layout, perm_host=None, tile_class_host=None) -> int:
+    """Fill host numpy arrays (perm int32 [S], tile classes uint8); return n_valid."""
+    nv = ctypes.c_int32(0)
+    pp = perm_host.ctypes.data if perm_host is not None else None
+    tp = tile_class_host.ctypes.data if tile_class_host is not None else None
+    _check(lib().h3_layout_export(layout.handle, pp, tp, ctypes.addressof(nv)),
+           "h3_layout_export")
+    return int(nv.value)
+
+
+def h3_workspace_size(dims: h3_dims, B: int, S: int) -> int:
+    return int(lib().h3_workspace_size(ctypes.byref(dims), B, S))
+
+
+def h3_pack_rows(layout: Layout, B: int, row_elems: int, video, audio, text, x_packed,
+                 stream=None) -> None:
+    _check(lib().h3_pack_rows(layout.handle, B, row_elems, _ptr(video), _ptr(audio), _ptr(text),
+                              _ptr(x_packed), _stream(stream)), "h3_pack_rows")
+
+
+def h3_unpack_rows(layout: Layout, B: int, row_elems: int, x_packed, video, audio, text,
+                   stream=None) -> None:
+    _check(lib().h3_unpack_rows(layout.handle, B, row_elems, _ptr(x_packed), _ptr(video),
+                                _ptr(audio), _ptr(text), _stream(stream)), "h3_unpack_rows")
+
+
+def h3_timestep_workspace_size(dims: h3_dims, n_t: int) -> int:
+    return int(lib().h3_timestep_workspace_size(ctypes.byref(dims), n_t))
+
+
+def h3_timestep_modulation(dims: h3_dims, n_t: int, t, w_t1, w_t2, w_proj, tmod, ws,
+                           ws_bytes: int, stream=None) -> None:
+    _check(lib().h3_timestep_modulation(ctypes.byref(dims), n_t, _ptr(t), _ptr(w_t1),
+                                        _ptr(w_t2), _ptr(w_proj), _ptr(tmod), _ptr(ws),
+                                        ws_bytes, _stream(stream)), "h3_timestep_modulation")
+
+
+def h3_norm_modulate(dims: h3_dims, layout: Layout, B: int, which: int, x, ada_table, tmod, h,
+                     stream=None) -> None:
+    _check(lib().h3_norm_modulate(ctypes.byref(dims), layout.handle, B, which, _ptr(x),
+                                  _ptr(ada_table), _ptr(tmod), _ptr(h), _stream(stream)),
+           "h3_norm_modulate")
+
+
+def h3_qkv_rope(dims: h3_dims, layout: Layout, B: int, h, w_qkv, q_norm, k_norm, q, k, v,
+                stream=None) -> None:
+    _check(lib().h3_qkv_rope(ctypes.byref(dims), layout.handle, B, _ptr(h), _ptr(w_qkv),
+                             _ptr(q_norm), _ptr(k_norm), _ptr(q), _ptr(k), _ptr(v),
+                             _stream(stream)), "h3_qkv_rope")
+
+
+def h3_attention(dims: h3_dims, layout: Layout, B: int, q, k, v, o, stream=None) -> None:
+    _check(lib().h3_attention(ctypes.byref(dims), layout.handle, B, _ptr(q), _ptr(k), _ptr(v),
+                              _ptr(o), _stream(stream)), "h3_attention")
+
+
+def h3_out_residual(dims: h3_dims, layout: Layout, B: int, o, w_o, ada_table, tmod, x,
+                    stream=None) -> None:
+    _check(lib().h3_out_residual(ctypes.byref(dims), layout.handle, B, _ptr(o), _ptr(w_o),
+                                 _ptr(ada_table), _ptr(tmod), _ptr(x), _stream(stream)),
+           "h3_out_residual")
+
+
+def h3_ffn_up(dims: h3_dims, layout: Layout, B: int, h2, w13, g, stream=None) -> None:
+    _check(lib().h3_ffn_up(ctypes.byref(dims), layout.handle, B, _ptr(h2), _ptr(w13), _ptr(g),
+                           _stream(stream)), "h3_ffn_up")
+
+
+def h3_ffn_down_residual(dims: h3_dims, layout: Layout, B: int, g, w2, ada_table, tmod, x,
+                         stream=None) -> None:
+    _check(lib().h3_ffn_down_residual(ctypes.byref(dims), layout.handle, B, _ptr(g), _ptr(w2),
+                                      _ptr(ada_table), _ptr(tmod), _ptr(x), _stream(stream)),
+           "h3_ffn_down_residual")
+
+
+def h3_block_forward(dims: h3_dims, weights: h3_block_weights, layout: Layout, tmod, x, B: int,
+                     ws, ws_bytes: int, stream=None) -> None:
+    _check(lib().h3_block_forward(ctypes.byref(dims), ctypes.byref(weights), layout.handle,
+                                  _ptr(tmod), _ptr(x), B, _ptr(ws), ws_bytes, _stream(stream)),
+           "h3_block_forward")
+
+
+def h3_stack_forward(dims: h3_dims, weights: Sequence[h3_block_weights], layout: Layout, tmod,
+                     x, B: int, ws, ws_bytes: int, stream=None) -> None:
+    arr = (h3_block_weights * max(1, len(weights)))(*weights)
+    _check(lib().h3_stack_forward(ctypes.byref(dims), arr, len(weights), layout.handle,
+                                  _ptr(tmod), _ptr(x), B, _ptr(ws), ws_bytes, _stream(stream)),
+           "h3_stack_forward")

@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark: packed rows/s of one MiniMax-H3 transformer-block forward on B200.
+
+Workload: the full-width single block over the 8192-row packed sequence
+(512 text | 6144 video rows of a (6, 32, 32) grid | 1536 audio rows, no
+padding), hidden 5376, 56 heads x 128, ffn 14336, one timestep per row,
+random-init bf16 weights ~N(0, 0.02) (synthetic data; no checkpoint).
+
+A step is one block forward (norm+modulate, QKV + QK-norm + RoPE, attention,
+O-projection + gated residual, norm+modulate, W1/W3 + SiLU gate, W2 + gated
+residual), in place on the packed hidden stream. The per-forward prologue
+(timestep MLP + AdaLN projection) and the layout step run once, before timing.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs under torch.distributed.run, one process per GPU; every rank runs
+its own replica of the workload (the batch axis is a pure replication axis,
+so there is no data-path collective) and the reported time is the maximum
+over ranks. ``--impl reference`` times the CPU oracle on a bounded sample of
+the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import (FULL_DIMS, activations, block_weights, config_layout,  # noqa: E402
+                       prologue_weights, make_layout)
+
+METRIC = "packed rows/s per DiT block fwd (bf16, 1xB200); % of dense bf16 TC peak"
+UNIT = "rows/s"
+CFG = 2
+WORKLOAD = ("full-width MiniMax-H3 block, S=8192 packed rows (512 text | 6144 video "
+            "(6,32,32) | 1536 audio), no padding, hidden 5376, 56x128 heads, ffn 14336, "
+            "per-row timesteps")
+KERNELS = ["norm_modulate_1", "qkv_rope", "attention", "out_residual", "norm_modulate_2",
+           "ffn_up", "ffn_down_residual"]
+
+
+# ------------------------------------------------------------------ work counts
+
+def kernel_work(dims, V):
+    """Algorithmic FLOPs (tensor kernels) or bytes (norm kernels) per launch."""
+    H, A, Fd, NH, D = dims.hidden, dims.attn_width, dims.ffn, dims.heads, dims.head_dim
+    norm_bytes = V * (2 * H + 2 * H + 2 * 4 * H)  # x in, h out, shift/scale rows of tmod (fp32)
+    return {
+        "norm_modulate_1": ("hbm", norm_bytes),
+        "qkv_rope": ("tensor", 2.0 * V * H * 3 * A),
+        "attention": ("tensor", 4.0 * NH * D * float(V) ** 2),
+        "out_residual": ("tensor", 2.0 * V * A * H),
+        "norm_modulate_2": ("hbm", norm_bytes),
+        "ffn_up": ("tensor", 2.0 * V * H * 2 * Fd),
+        "ffn_down_residual": ("tensor", 2.0 * V * Fd * H),
+    }
+
+
+def block_flops(dims, V):
+    return sum(v for k, (b, v) in kernel_work(dims, V).items() if b == "tensor")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Maximum of a float over all ranks (identity for a single process)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None) -> None:
+    if world <= 1:
+        return
+    import torch.distributed as dist
+    if device is not None and dist.get_backend() == "nccl":
+        dist.barrier(device_ids=[device.index])
+    else:
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_sample(rows: int = 512):
+    """Time the oracle on the first ``rows`` text-like rows as a packed sequence of
+    their own; report rows/s scaled to the full workload's per-row work."""
+    from oracle import h3_oracle as O  # CPU baseline only
+    dims = FULL_DIMS
+    w = block_weights(dims, CFG, 0)
+    L = make_layout([("text", 0, rows)], seed=[CFG])
+    x = O.bf16_to_f64(activations(dims, CFG, rows))
+    pw = prologue_weights(dims, CFG)
+    t0 = time.perf_counter()
+    tm = O.timestep_modulation(L.timestep, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim,
+                               dims.hidden)
+    t1 = time.perf_counter()
+    O.block_forward(x, w, L, tm, dims)
+    t2 = time.perf_counter()
+    full_S = config_layout(CFG).S
+    per_row_sample = block_flops(dims, rows) / rows
+    per_row_full = block_flops(dims, full_S) / full_S
+    rate = rows / (t2 - t1) * (per_row_sample / per_row_full)
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    return {
+        "value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+        "sample": (f"float64 NumPy oracle block forward on {rows} packed rows as their own "
+                   f"sequence ({t2 - t1:.2f} s; prologue {t1 - t0:.2f} s not counted), rows/s "
+                   f"scaled by per-row work {per_row_sample / 1e6:.0f} / "
+                   f"{per_row_full / 1e6:.0f} MFLOP to the {full_S}-row workload"),
+    }
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: each step is one bounded CPU sample of the
+    workload; the run is time-boxed so that it ends within a few minutes."""
+    if rank != 0:
+        return 0
+    per = []
+    oracle_sample(args.ref_rows)  # one untimed warm-up sample (BLAS threads, caches)
+    t0 = time.perf_counter()
+    for _ in range(max(1, args.steps)):
+        per.append(oracle_sample(args.ref_rows))
+        if time.perf_counter() - t0 > args.ref_budget_s:
+            break
+    val = statistics.median(p["value"] for p in per)
+    base = per[0]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "samples_run": len(per),
+        "ms_per_step": config_layout(CFG).S / val * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "S": config_layout(CFG).S, "B": 1},
+        "cpu_baseline": dict(base, value=val),
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, world, rank, local):
+    import torch
+    from audio_generation_b200 import h3
+
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dims = FULL_DIMS
+    d = h3.make_dims(dims)
+    L = config_layout(CFG)
+    S, V, B = L.S, L.n_valid, 1
+
+    def to_dev_bits(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(
+            torch.bfloat16)
+
+    def to_dev_f32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+    def to_dev_i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+    w = block_weights(dims, CFG, 0)
+    pw = prologue_weights(dims, CFG)
+    wd = {k: to_dev_bits(getattr(w, k)) for k in ("w_qkv", "q_norm", "k_norm", "w_o", "w13", "w2")}
+    wd["ada_table"] = to_dev_f32(w.ada_table)
+    cw = h3.make_block_weights(wd["w_qkv"], wd["q_norm"], wd["k_norm"], wd["w_o"], wd["w13"],
+                               wd["w2"], wd["ada_table"])
+    pos, tags, tidx = to_dev_f32(L.pos), to_dev_i32(L.tags), to_dev_i32(L.t_idx)
+    vi, ai, ti = to_dev_i32(L.video_idx), to_dev_i32(L.audio_idx), to_dev_i32(L.text_idx)
+    layout = h3.h3_layout_prepare(d, S, L.n_t, pos, tags, tidx, vi, ai, ti)
+    # per-forward prologue: tmod for the per-row timesteps
+    tws_b = h3.h3_timestep_workspace_size(d, L.n_t)
+    tws = torch.empty(tws_b, dtype=torch.uint8, device=device)
+    tmod = torch.empty((L.n_t, 6, dims.hidden), dtype=torch.float32, device=device)
+    h3.h3_timestep_modulation(d, L.n_t, to_dev_f32(L.timestep), to_dev_f32(pw.w_t1),
+                              to_dev_f32(pw.w_t2), to_dev_f32(pw.w_proj), tmod, tws, tws_b)
+    del tws
+    x_host = torch.from_numpy(activations(dims, CFG, S, B).view(np.int16)).view(
+        torch.bfloat16).pin_memory()
+    x = x_host.to(device)
+    ws_b = h3.h3_workspace_size(d, B, S)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        h3.h3_block_forward(d, cw, layout, tmod, x, B, ws, ws_b, stream)
+
+    # ---- whole-step timing (device events, max over ranks)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    gpu_id = torch.cuda.get_device_properties(device).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(gpu_id) as clk:
+        time.sleep(0.3)  # let the sampler start before the timed region
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world, device)
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world, device)
+    err = h3.h3_layout_error(layout)
+    if err != h3.H3_OK:
+        raise RuntimeError(f"device error word after timing: {h3.h3_status_string(err)}")
+    ms_per_step = ms / args.steps
+    value = world * B * S / (ms_per_step / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    out_host = torch.empty_like(x_host).pin_memory()
+    for _ in range(2):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        out_host.copy_(x, non_blocking=True)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        out_host.copy_(x, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / args.steps
+    io_bytes = x_host.numel() * 2
+
+    # ---- per-kernel device time inside a run of steps (for the roofline)
+    per = {k: 0.0 for k in KERNELS}
+    h, g = ws, None  # workspace views for the single steps
+    A, Fd = dims.attn_width, dims.ffn
+    hbuf = torch.empty((B, S, dims.hidden), dtype=torch.bfloat16, device=device)
+    q = torch.empty((B, dims.heads, S, 128), dtype=torch.bfloat16, device=device)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    o = torch.empty((B, S, A), dtype=torch.bfloat16, device=device)
+    gbuf = torch.empty((B, S, Fd), dtype=torch.bfloat16, device=device)
+    launches = [
+        ("norm_modulate_1", lambda: h3.h3_norm_modulate(d, layout, B, 0, x, wd["ada_table"], tmod, hbuf, stream)),
+        ("qkv_rope", lambda: h3.h3_qkv_rope(d, layout, B, hbuf, wd["w_qkv"], wd["q_norm"], wd["k_norm"], q, k, v, stream)),
+        ("attention", lambda: h3.h3_attention(d, layout, B, q, k, v, o, stream)),
+        ("out_residual", lambda: h3.h3_out_residual(d, layout, B, o, wd["w_o"], wd["ada_table"], tmod, x, stream)),
+        ("norm_modulate_2", lambda: h3.h3_norm_modulate(d, layout, B, 1, x, wd["ada_table"], tmod, hbuf, stream)),
+        ("ffn_up", lambda: h3.h3_ffn_up(d, layout, B, hbuf, wd["w13"], gbuf, stream)),
+        ("ffn_down_residual", lambda: h3.h3_ffn_down_residual(d, layout, B, gbuf, wd["w2"], wd["ada_table"], tmod, x, stream)),
+    ]
+    reps = max(3, min(20, args.steps))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)]
+           for _ in range(reps)]
+    for _, fn in launches:
+        fn()
+    for r in range(reps):
+        evs[r][0].record(stream)
+        for i, (_, fn) in enumerate(launches):
+            fn()
+            evs[r][i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    for r in range(reps):
+        for i, (name, _) in enumerate(launches):
+            per[name] += evs[r][i].elapsed_time(evs[r][i + 1]) / reps
+    work = kernel_work(dims, V)
+    peaks = load_peaks()
+    dom = max(per, key=lambda n: per[n])
+    bound, amount = work[dom]
+    if bound == "tensor":
+        achieved = amount / (per[dom] * 1e-3) / 1e12
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved = amount / (per[dom] * 1e-3) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    kernels = {}
+    for n in KERNELS:
+        b, amt = work[n]
+        t = per[n] * 1e-3
+        if b == "tensor":
+            kernels[n] = {"ms": round(per[n], 4), "tflops": round(amt / t / 1e12, 1),
+                          "frac_of_peak": round(amt / t / 1e12 / peaks["bf16_tflops"], 3)}
+        else:
+            kernels[n] = {"ms": round(per[n], 4), "gbs": round(amt / t / 1e9, 1),
+                          "frac_of_peak": round(amt / t / 1e9 / peaks["hbm_gbs"], 3)}
+    flops = block_flops(dims, V)
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights and activations)",
+        "config": {"workload": WORKLOAD, "S": S, "B": B, "valid_rows": V,
+                   "l2": "inputs larger than L2 (770 MB of block weights + 1 GB tmod per step)",
+                   "parallelism": f"replicas x{world}, no collective on the data path"},
+        "tflops": flops / (ms_per_step * 1e-3) / 1e12,
+        "frac_of_peak": flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "peak_source": peaks["source"],
+        "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
+                     "unit": unit, "frac": achieved / peak, "traffic": None},
+        "kernels": kernels,
+        "e2e": {"value": world * B * S / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
+        "gpu_launches": len(launches) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(args.ref_rows)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    layout.close()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--ref-rows", type=int, default=512,
+                    help="rows of the oracle's bounded CPU sample")
+    ap.add_argument("--ref-budget-s", type=float, default=150.0,
+                    help="time box of the reference arm's timed samples")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_gpu(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

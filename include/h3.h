@@ -1,0 +1,246 @@
+/*
+ * h3.h — C ABI of the B200 (sm_100a) MiniMax-H3 transformer-block library.
+ *
+ * What the library computes is defined on the page "MiniMaxH3Transformer3DModel"
+ * (diffusers v0.43.0 docs): one stack of blocks runs over a single packed 1-D
+ * sequence of text, conditioning, audio and target-video rows; attention is
+ * full self-attention over that sequence; the per-row modality tag selects the
+ * AdaLN modulation; rows tagged -1 (padding) form their own attention document
+ * under a boolean mask; the caller builds the packing and passes the layout
+ * (the (t, h, w) grid, per-row tags, per-row timestep indices and the three
+ * index tensors) separately from the latents (section "MiniMaxH3Transformer3DModel",
+ * constructor parameters and `forward` arguments). The block structure follows
+ * the same page's constructor parameters and the page "MiniMax H3 Inference
+ * Engine voor Mac computers", sections "Exacte DiT fusions" (gated attention
+ * residual feeding the MLP's AdaLN over a bf16 residual stream), "Checkpoint
+ * layout en media pipeline" (QKV rows interleaved per head, fused
+ * QK-norm + RoPE) and "Profiling en diagnostische pads" (fc1 -> SwiGLU -> fc2).
+ *
+ * Conventions shared by every entry point:
+ *  - Ownership: the caller owns every buffer. Pointers named in structs and
+ *    arguments are DEVICE pointers unless the name ends in `_host`. The library
+ *    allocates device memory only in h3_layout_prepare (small per-layout tables,
+ *    released by h3_layout_destroy).
+ *  - Types: "bf16" buffers hold IEEE bfloat16 values (2 bytes each); "f32"
+ *    buffers hold float; index buffers hold int32_t.
+ *  - Matrices are row-major [out, in] (K-major for the tensor cores).
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *    default stream). Every call except h3_layout_prepare, h3_layout_error and
+ *    h3_layout_export only enqueues work and returns; argument, shape and
+ *    alignment errors are returned synchronously before anything is launched.
+ *  - Alignment: every device pointer must be 16-byte aligned.
+ *  - Shapes: head_dim == 128; hidden % 256 == 0; heads even; ffn % 128 == 0;
+ *    rope_freq_dim == 16; time dims % 4 == 0. S (rows) is arbitrary >= 0.
+ *  - Batch: B >= 1 elements share one layout; each element is its own attention
+ *    document set (the page's "pure replication axis").
+ *  - Asynchronous failures: every wait inside a kernel is bounded (about 2 s).
+ *    A wait that runs out records an error in the layout's device error word;
+ *    read it with h3_layout_error after the stream has been synchronised.
+ */
+#ifndef H3_H
+#define H3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define H3_API __attribute__((visibility("default")))
+#else
+#define H3_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  H3_OK = 0,
+  H3_ERR_ARG = -1,       /* null pointer, negative size, unknown option */
+  H3_ERR_SHAPE = -2,     /* dimensions the kernels do not support */
+  H3_ERR_ALIGN = -3,     /* pointer not 16-byte aligned */
+  H3_ERR_LAYOUT = -4,    /* layout tensors inconsistent (see h3_layout_prepare) */
+  H3_ERR_WORKSPACE = -5, /* workspace smaller than h3_workspace_size */
+  H3_ERR_CUDA = -6,      /* a CUDA runtime/driver call failed */
+  H3_ERR_TIMEOUT = -7    /* a bounded in-kernel wait ran out */
+} h3_status;
+
+typedef void* h3_stream_t;
+
+/* Block dimensions: the constructor parameters of the transformer
+ * (num_attention_heads, attention_head_dim, hidden_size, ffn_dim,
+ * time_embed_dim, time_embed_hidden_dim, freq_dim, rope_freq_dim, rope_theta,
+ * norm_eps, qk_norm_eps). n_modalities is the number of AdaLN table rows (3:
+ * video 0, text 1, audio 2). */
+typedef struct {
+  int hidden, heads, head_dim, ffn, time_embed_dim, time_hidden, freq_dim, rope_freq_dim,
+      n_modalities;
+  float rope_theta, norm_eps, qk_norm_eps;
+} h3_dims;
+
+/* The packed layout, as the `forward` arguments describe it. All DEVICE
+ * pointers; read only during h3_layout_prepare (the library keeps copies).
+ *   pos       [S, 3] f32  (t, h, w) rotary coordinates; fp32 so that halved
+ *                         (fractional) spatial coordinates are representable
+ *   tags      [S]    i32  0 video, 1 text, 2 audio, -1 padding
+ *   t_idx     [S]    i32  index of the row's value in `timestep` (0 <= t_idx < n_t)
+ *   video_idx [n_video], audio_idx [n_audio], text_idx [n_text]  i32:
+ *             packed-row positions of the rows of each modality, in the order of
+ *             that modality's latent rows. */
+typedef struct {
+  int S, n_t, n_video, n_audio, n_text;
+  const float* pos;
+  const int32_t* tags;
+  const int32_t* t_idx;
+  const int32_t* video_idx;
+  const int32_t* audio_idx;
+  const int32_t* text_idx;
+} h3_layout_desc;
+
+typedef struct h3_layout* h3_layout_t;
+
+/* One block's parameters (DEVICE pointers, [out, in] row-major):
+ *   w_qkv     [3*NH*D, H] bf16, rows interleaved per head: row n*3D + {0, D, 2D} + d
+ *             holds q / k / v channel d of head n
+ *   q_norm, k_norm [D] bf16  per-head RMSNorm weights (shared by all heads)
+ *   w_o       [H, NH*D] bf16
+ *   w13       [2F, H] bf16, W1 and W3 interleaved in 128-row blocks:
+ *             rows [256j, 256j+128) = W1 rows [128j, 128j+128),
+ *             rows [256j+128, 256j+256) = W3 rows [128j, 128j+128)
+ *   w2        [H, F] bf16
+ *   ada_table [n_modalities, 6, H] f32: per-modality AdaLN rows in the order
+ *             (shift1, scale1, gate1, shift2, scale2, gate2) */
+typedef struct {
+  const void* w_qkv;
+  const void* q_norm;
+  const void* k_norm;
+  const void* w_o;
+  const void* w13;
+  const void* w2;
+  const float* ada_table;
+} h3_block_weights;
+
+/* Human-readable name of a status code (static string). */
+H3_API const char* h3_status_string(h3_status status);
+
+/* Library ABI version (increases when a signature changes). */
+H3_API int h3_abi_version(void);
+
+/* a0 — validate a packed layout and build its device tables: per-128-row tile
+ * classes (all valid / all padding / mixed), the valid-key bitmask of each
+ * tile, the compaction order (valid rows first, then padding rows, each in
+ * packed order), the per-row source of the packing, and the per-row RoPE
+ * cos/sin table (inv_freq[j] = rope_theta^(-j/rope_freq_dim)).
+ * Validation (all on the GPU): tags in {-1,0,1,2}; every t_idx in [0, n_t);
+ * positions finite; every index tensor in range, duplicate-free, pointing
+ * only at rows of its modality and as long as the number of such rows.
+ * Synchronises `stream` once. On H3_ERR_LAYOUT nothing is returned in *out.
+ * The layout object owns a device error word used by the later calls. */
+H3_API h3_status h3_layout_prepare(const h3_dims* dims, const h3_layout_desc* desc, h3_stream_t stream,
+                            h3_layout_t* out);
+
+/* Release a layout (synchronises the device first). NULL is ignored. */
+H3_API void h3_layout_destroy(h3_layout_t layout);
+
+/* Read and clear the layout's device error word (synchronises the device):
+ * H3_OK, or H3_ERR_TIMEOUT if a bounded in-kernel wait ran out. */
+H3_API h3_status h3_layout_error(h3_layout_t layout);
+
+/* Copy the layout's tables to HOST buffers (any may be NULL):
+ * perm_host [S] compaction order, tile_class_host [ceil(S/128)] (0 valid,
+ * 1 padding, 2 mixed), n_valid_host [1]. Synchronous. */
+H3_API h3_status h3_layout_export(h3_layout_t layout, int32_t* perm_host, uint8_t* tile_class_host,
+                           int32_t* n_valid_host);
+
+/* Bytes of device workspace h3_block_forward / h3_stack_forward need for B
+ * batch elements of S rows. 0 on invalid dims. */
+H3_API size_t h3_workspace_size(const h3_dims* dims, int B, int S);
+
+/* a1 — scatter per-modality rows into the packed stream (bit-exact copies):
+ * x_packed[b, video_idx[i]] = video[b, i] (same for audio and text); padding
+ * rows are zero-filled. Rows are `row_elems` bf16 values wide; video [B, n_video,
+ * row_elems], audio [B, n_audio, row_elems], text [B, n_text, row_elems],
+ * x_packed [B, S, row_elems]. row_elems % 8 == 0. */
+H3_API h3_status h3_pack_rows(h3_layout_t layout, int B, int row_elems, const void* video,
+                       const void* audio, const void* text, void* x_packed, h3_stream_t stream);
+
+/* a1 — gather packed rows back to per-modality buffers (bit-exact), in index
+ * order (the page's `forward` returns velocities in the row order of
+ * video_indices and audio_indices). Any output may be NULL to skip it. */
+H3_API h3_status h3_unpack_rows(h3_layout_t layout, int B, int row_elems, const void* x_packed,
+                         void* video, void* audio, void* text, h3_stream_t stream);
+
+/* a2 — timestep embedding and shared AdaLN projection, fp32 throughout:
+ * tmod[n, 6H] = W_proj . SiLU(W_t2 . SiLU(W_t1 . [cos(t f_i), sin(t f_i)])),
+ * f_i = 10^4^(-i/(freq_dim/2)); timesteps unscaled in [0, 1] (constructor
+ * parameters freq_dim, time_embed_hidden_dim, time_embed_dim).
+ *   t [n_t] f32, w_t1 [time_hidden, freq_dim], w_t2 [time_embed_dim, time_hidden],
+ *   w_proj [6H, time_embed_dim] (all f32), tmod [n_t, 6, H] f32.
+ * ws must hold h3_timestep_workspace_size(dims, n_t) bytes. */
+H3_API size_t h3_timestep_workspace_size(const h3_dims* dims, int n_t);
+H3_API h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const float* t, const float* w_t1,
+                                 const float* w_t2, const float* w_proj, float* tmod, void* ws,
+                                 size_t ws_bytes, h3_stream_t stream);
+
+/* ---- single steps of the block (each also runs inside h3_block_forward) ---- */
+
+/* a3 / a7 — h = LayerNorm(x) * (1 + scale) + shift (no affine, biased
+ * variance, eps = norm_eps), with shift/scale of row r = ada_table[tag(r)][c]
+ * + tmod[t_idx(r)][c] for c = (shift, scale) = (0, 1) when which == 0 and
+ * (3, 4) when which == 1. x, h [B, S, H] bf16; padding rows of h are zero. */
+H3_API h3_status h3_norm_modulate(const h3_dims* dims, h3_layout_t layout, int B, int which,
+                           const void* x, const float* ada_table, const float* tmod, void* h,
+                           h3_stream_t stream);
+
+/* a4 — qkv = h . W_qkv^T on tcgen05; per head: q, k <- RMSNorm(., q_norm/k_norm,
+ * qk_norm_eps), then RoPE on channels [0, 96): pair (32a + j, 32a + j + 16),
+ * a = (t, h, w), angle pos[r][a] * inv_freq[j]. q, k, v [B, NH, S, D] bf16. */
+H3_API h3_status h3_qkv_rope(const h3_dims* dims, h3_layout_t layout, int B, const void* h,
+                      const void* w_qkv, const void* q_norm, const void* k_norm, void* q,
+                      void* k, void* v, h3_stream_t stream);
+
+/* a5 — o = softmax(q k^T / sqrt(D)) v per head over the row's document
+ * (valid rows attend valid rows; padding query rows are not computed and
+ * their output rows are zero). q, k, v [B, NH, S, D] bf16 -> o [B, S, NH*D] bf16. */
+H3_API h3_status h3_attention(const h3_dims* dims, h3_layout_t layout, int B, const void* q,
+                       const void* k, const void* v, void* o, h3_stream_t stream);
+
+/* a6 — x += gate1 * (o . W_o^T) in place, gate1 = ada_table[tag][2] + tmod[t_idx][2];
+ * padding rows of x are left untouched. o [B, S, NH*D] bf16, x [B, S, H] bf16. */
+H3_API h3_status h3_out_residual(const h3_dims* dims, h3_layout_t layout, int B, const void* o,
+                          const void* w_o, const float* ada_table, const float* tmod, void* x,
+                          h3_stream_t stream);
+
+/* a8 — g = SiLU(h2 . W1^T) * (h2 . W3^T) from the block-interleaved w13.
+ * h2 [B, S, H] bf16 -> g [B, S, F] bf16. */
+H3_API h3_status h3_ffn_up(const h3_dims* dims, h3_layout_t layout, int B, const void* h2,
+                    const void* w13, void* g, h3_stream_t stream);
+
+/* a9 — x += gate2 * (g . W2^T) in place, gate2 = ada_table[tag][5] + tmod[t_idx][5];
+ * padding rows untouched. g [B, S, F] bf16, x [B, S, H] bf16. */
+H3_API h3_status h3_ffn_down_residual(const h3_dims* dims, h3_layout_t layout, int B, const void* g,
+                               const void* w2, const float* ada_table, const float* tmod,
+                               void* x, h3_stream_t stream);
+
+/* ---- the block and the stack ---- */
+
+/* One block, in place on x [B, S, H] bf16: a3, a4, a5, a6, a7, a8, a9 with
+ * tmod [n_t, 6, H] f32 (from h3_timestep_modulation). Padding rows of x are
+ * returned bit-identical. ws: h3_workspace_size(dims, B, S) bytes. */
+H3_API h3_status h3_block_forward(const h3_dims* dims, const h3_block_weights* weights,
+                           h3_layout_t layout, const float* tmod, void* x, int B, void* ws,
+                           size_t ws_bytes, h3_stream_t stream);
+
+/* n_blocks blocks (weights: HOST array of n_blocks structs holding device
+ * pointers) sharing one tmod, in place on x [B, S, H] bf16. Valid rows are
+ * gathered once into a compact [B, V, H] stream (padding rows never reach a
+ * valid row's result, so the blocks then run with no mask), and scattered back
+ * at the end; padding rows of x are untouched. */
+H3_API h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* weights, int n_blocks,
+                           h3_layout_t layout, const float* tmod, void* x, int B, void* ws,
+                           size_t ws_bytes, h3_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3_H */

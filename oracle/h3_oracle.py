@@ -280,14 +280,16 @@ def block_forward(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
     return out
 
 
-def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable[[np.ndarray], np.ndarray],
-                       dims, rows: np.ndarray, chunk: int = 2048) -> np.ndarray:
+def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable, dims, rows: np.ndarray,
+                       chunk: int = 2048) -> np.ndarray:
     """The same block evaluated only at the query rows ``rows`` (B = 1).
 
     Keys and values are needed for every row, so they are formed for all rows
-    in row chunks (each row's k and v depend on that row alone). ``tmod_rows``
-    maps timestep indices to their tmod rows [n, 6, H], so a caller with one
-    timestep per row never holds tmod for the whole sequence.
+    in row chunks (each row's k and v depend on that row alone).
+    ``tmod_rows(t_idx, n_chunks)`` returns the first ``n_chunks`` modulation
+    chunks of tmod for those timestep indices, [n, n_chunks, H]: the key/value
+    pass asks only for (shift1, scale1), so a caller with one timestep per row
+    never forms the whole tmod.
     """
     x = np.asarray(x, F)
     S = x.shape[0]
@@ -297,13 +299,14 @@ def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable[[np.ndarray
     K = np.empty((S, NH, D), F)
     V = np.empty((S, NH, D), F)
     table = np.asarray(w.ada_table, F)
+    t_idx = np.asarray(layout.t_idx)
     for r0 in range(0, S, chunk):
         r1 = min(S, r0 + chunk)
         tg = tags[r0:r1]
-        m = np.zeros((r1 - r0, 6, dims.hidden), F)
+        m = np.zeros((r1 - r0, 2, dims.hidden), F)
         vv = tg >= 0
         if vv.any():
-            m[vv] = table[tg[vv]] + tmod_rows(np.asarray(layout.t_idx)[r0:r1][vv])
+            m[vv] = table[tg[vv], :2] + tmod_rows(t_idx[r0:r1][vv], 2)
         _, K[r0:r1], V[r0:r1] = _pre_attention(x[r0:r1], m, layout.pos[r0:r1], w, dims,
                                                False, need_q=False)
     rows = np.asarray(rows)
@@ -311,7 +314,7 @@ def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable[[np.ndarray
     m = np.zeros((rows.shape[0], 6, dims.hidden), F)
     vv = tg >= 0
     if vv.any():
-        m[vv] = table[tg[vv]] + tmod_rows(np.asarray(layout.t_idx)[rows][vv])
+        m[vv] = table[tg[vv]] + tmod_rows(t_idx[rows][vv], 6)
     q, _, _ = _pre_attention(x[rows], m, layout.pos[rows], w, dims, False)
     o = attention(q, pad[rows], K, V, pad)
     y = _post_attention(x[rows], o, m, w, dims, False)

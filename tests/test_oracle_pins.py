@@ -478,7 +478,7 @@ def test_block_rows_evaluator_matches_full_block():
     L, w, x, tmod = _small_case(S=70, seed=6)
     y = O.block_forward(x, w, L, tmod, SMALL)
     rows = np.array([0, 5, 17, 33, 69])
-    yr = O.block_forward_rows(x[0], w, L, lambda ti: tmod[ti], SMALL, rows, chunk=16)
+    yr = O.block_forward_rows(x[0], w, L, lambda ti, c: tmod[ti, :c], SMALL, rows, chunk=16)
     np.testing.assert_allclose(yr, y[0, rows], rtol=1e-12, atol=1e-12)
 
 

@@ -121,10 +121,10 @@ class PrologueWeights:
 # --------------------------------------------------------------------------
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
-    """Round float32 values to bf16 (nearest, ties to even); return uint16 bits."""
+    """Round finite float32 values to bf16 (nearest, ties to even); return uint16 bits."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    u = a.view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return r.astype(np.uint16)
 
 
@@ -144,10 +144,10 @@ def _threads() -> int:
         return os.cpu_count() or 1
 
 
-def _normal_f32(shape: Tuple[int, ...], seed: Sequence[int], std: float,
-                mean: float = 0.0) -> np.ndarray:
+def _normal_chunks(shape: Tuple[int, ...], seed: Sequence[int], std: float, mean: float,
+                   to_bf16: bool) -> np.ndarray:
     n = int(np.prod(shape)) if len(shape) else 1
-    out = np.empty(n, dtype=np.float32)
+    out = np.empty(n, dtype=np.uint16 if to_bf16 else np.float32)
     n_chunks = (n + _CHUNK - 1) // _CHUNK
 
     def fill(i: int) -> None:
@@ -158,7 +158,7 @@ def _normal_f32(shape: Tuple[int, ...], seed: Sequence[int], std: float,
             v *= np.float32(std)
         if mean != 0.0:
             v += np.float32(mean)
-        out[lo:hi] = v
+        out[lo:hi] = f32_to_bf16_bits(v) if to_bf16 else v
 
     if n_chunks <= 1:
         for i in range(n_chunks):
@@ -169,10 +169,15 @@ def _normal_f32(shape: Tuple[int, ...], seed: Sequence[int], std: float,
     return out.reshape(shape)
 
 
+def _normal_f32(shape: Tuple[int, ...], seed: Sequence[int], std: float,
+                mean: float = 0.0) -> np.ndarray:
+    return _normal_chunks(shape, seed, std, mean, False)
+
+
 def normal_bf16(shape: Tuple[int, ...], seed: Sequence[int], std: float = 1.0,
                 mean: float = 0.0) -> np.ndarray:
     """N(mean, std^2) draws rounded to bf16; returns uint16 bit patterns."""
-    return f32_to_bf16_bits(_normal_f32(tuple(shape), seed, std, mean)).reshape(shape)
+    return _normal_chunks(tuple(shape), seed, std, mean, True)
 
 
 def normal_f32(shape: Tuple[int, ...], seed: Sequence[int], std: float = 1.0) -> np.ndarray:
