@@ -57,7 +57,7 @@ size_t ws_parts(const h3_dims& d, int B, int S, Workspace* w, void* base) {
   const size_t g_b = align256(rows * (size_t)d.ffn * 2);  // g reuses the q/k/v region
   const size_t qg_b = 3 * one_b > g_b ? 3 * one_b : g_b;
   const size_t o_b = align256(rows * A * 2);
-  const size_t xc_b = align256(rows * d.hidden * 2);
+  const size_t xc_b = align256(rows * d.hidden * 4);  // the stack's fp32 residual stream
   if (w) {
     uint8_t* p = static_cast<uint8_t*>(base);
     w->h = p;
@@ -82,13 +82,16 @@ h3_status check_weights(const h3_block_weights* w) {
   return H3_OK;
 }
 
-// One block over the rows described by `L` (full or compacted view), in place on x.
+// One block over the rows described by `L` (full or compacted view), in place on
+// x: bf16 for h3_block_forward, fp32 (x_f32) for the stack's residual stream.
 h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutView& L,
-                    const float* tmod, void* x, int B, const Workspace& ws, cudaStream_t st) {
+                    const float* tmod, void* x, bool x_f32, int B, const Workspace& ws,
+                    cudaStream_t st) {
   const int M = B * L.S;
   if (M == 0) return H3_OK;
   const int H = d.hidden, A = d.heads * d.head_dim, Fd = d.ffn;
-  H3_CUDA(launch_norm_modulate(L, B, H, 0, 1, d.norm_eps, x, w.ada_table, tmod, ws.h, st));
+  H3_CUDA(launch_norm_modulate(L, B, H, 0, 1, d.norm_eps, x, x_f32, w.ada_table, tmod, ws.h,
+                               st));
   GemmEpiArgs e;
   e.L = L;
   e.B = B;
@@ -108,14 +111,16 @@ h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutVie
   r.table = w.ada_table;
   r.tmod = tmod;
   r.gate_chunk = 2;
-  H3_CUDA(launch_gemm(EPI_RESID, M, H, A, ws.o, w.w_o, r, st));
-  H3_CUDA(launch_norm_modulate(L, B, H, 3, 4, d.norm_eps, x, w.ada_table, tmod, ws.h, st));
+  const int resid = x_f32 ? EPI_RESID_F32 : EPI_RESID;
+  H3_CUDA(launch_gemm(resid, M, H, A, ws.o, w.w_o, r, st));
+  H3_CUDA(launch_norm_modulate(L, B, H, 3, 4, d.norm_eps, x, x_f32, w.ada_table, tmod, ws.h,
+                               st));
   GemmEpiArgs sg;
   sg.L = L;
   sg.out = ws.g;
   H3_CUDA(launch_gemm(EPI_SWIGLU, M, 2 * Fd, H, ws.h, w.w13, sg, st));
   r.gate_chunk = 5;
-  H3_CUDA(launch_gemm(EPI_RESID, M, H, Fd, ws.g, w.w2, r, st));
+  H3_CUDA(launch_gemm(resid, M, H, Fd, ws.g, w.w2, r, st));
   return H3_OK;
 }
 
@@ -337,7 +342,7 @@ h3_status h3_norm_modulate(const h3_dims* dims, h3_layout_t L, int B, int which,
   if (!aligned16(x) || !aligned16(ada_table) || !aligned16(tmod) || !aligned16(h))
     return H3_ERR_ALIGN;
   const int c0 = which == 0 ? 0 : 3;
-  H3_CUDA(launch_norm_modulate(L->view(), B, dims->hidden, c0, c0 + 1, dims->norm_eps, x,
+  H3_CUDA(launch_norm_modulate(L->view(), B, dims->hidden, c0, c0 + 1, dims->norm_eps, x, false,
                                ada_table, tmod, h, as_stream(stream)));
   return H3_OK;
 }
@@ -436,7 +441,7 @@ h3_status h3_block_forward(const h3_dims* dims, const h3_block_weights* weights,
   if (ws_bytes < h3_workspace_size(dims, B, L->S)) return H3_ERR_WORKSPACE;
   Workspace w;
   ws_parts(*dims, B, L->S, &w, ws);
-  return run_block(*dims, *weights, L->view(), tmod, x, B, w, as_stream(stream));
+  return run_block(*dims, *weights, L->view(), tmod, x, false, B, w, as_stream(stream));
 }
 
 h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* weights, int n_blocks,
@@ -451,18 +456,15 @@ h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* weights,
   cudaStream_t st = as_stream(stream);
   Workspace w;
   ws_parts(*dims, B, L->S, &w, ws);
-  if (L->n_valid == L->S) {
-    for (int i = 0; i < n_blocks; ++i)
-      H3_TRY(run_block(*dims, weights[i], L->view(), tmod, x, B, w, st));
-    return H3_OK;
-  }
-  // Valid rows never see padding rows, and padding rows leave every block
-  // unchanged, so the blocks run on the compacted valid rows alone.
+  // The valid rows are gathered once (in packed order, padding rows dropped:
+  // they never reach a valid row's result and every block leaves them
+  // unchanged) into an fp32 residual stream, which all blocks update; the
+  // result is rounded to bf16 once when it is scattered back.
   const int V = L->n_valid;
-  H3_CUDA(launch_permute_rows(B, V, L->S, dims->hidden, L->perm, x, w.xc, true, st));
+  H3_CUDA(launch_permute_rows_convert(B, V, L->S, dims->hidden, L->perm, x, w.xc, true, st));
   for (int i = 0; i < n_blocks; ++i)
-    H3_TRY(run_block(*dims, weights[i], L->compact_view(), tmod, w.xc, B, w, st));
-  H3_CUDA(launch_permute_rows(B, V, L->S, dims->hidden, L->perm, w.xc, x, false, st));
+    H3_TRY(run_block(*dims, weights[i], L->compact_view(), tmod, w.xc, true, B, w, st));
+  H3_CUDA(launch_permute_rows_convert(B, V, L->S, dims->hidden, L->perm, w.xc, x, false, st));
   return H3_OK;
 }
 

@@ -21,7 +21,8 @@
 //              channel pairs (32a + j, 32a + j + 16); stores head-major
 //              [B, NH, S, 128] bf16.
 //   EPI_RESID  x <- x + gate * acc (gated residual, "Exacte DiT fusions"),
-//              gate = ada_table[tag][c] + tmod[t_idx][c]; padding rows skipped.
+//              gate = ada_table[tag][c] + tmod[t_idx][c]; padding rows skipped;
+//              x bf16 (EPI_RESID) or fp32 (EPI_RESID_F32, the stack's stream).
 //   EPI_SWIGLU W1 / W3 interleaved in 128-row blocks: g = SiLU(a) * b.
 //   EPI_STORE  plain bf16 store (the GEMM core on its own).
 #include "host_util.cuh"
@@ -98,12 +99,11 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
       for (int i = 0; i < 32; ++i) a[i] = a[i] / (1.f + __expf(-a[i])) * b[i];
       if (row_ok) store_bf16x32(out + (size_t)m * ldo + n0 / 2 + 32 * c, a);
     }
-  } else if constexpr (EPI == EPI_RESID) {
+  } else if constexpr (EPI == EPI_RESID || EPI == EPI_RESID_F32) {
     const int s = row_ok ? m % e.L.S : 0;
     const int tag = row_ok ? e.L.tags[s] : -1;
     const int ti = row_ok ? e.L.t_idx[s] : 0;
     const bool active = row_ok && tag >= 0;
-    __nv_bfloat16* x = reinterpret_cast<__nv_bfloat16*>(e.x);
     const float* gt = e.table + ((size_t)(active ? tag : 0) * 6 + e.gate_chunk) * N + n0;
     const float* gm = e.tmod + ((size_t)ti * 6 + e.gate_chunk) * N + n0;
 #pragma unroll 1
@@ -111,9 +111,18 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
       float v[32];
       ld_acc(taddr + 32 * c, v);
       if (active) {
-        __nv_bfloat16* xp = x + (size_t)m * N + n0 + 32 * c;
         float xv[32];
-        load_bf16x32(xp, xv);
+        const size_t off = (size_t)m * N + n0 + 32 * c;
+        if constexpr (EPI == EPI_RESID) {
+          load_bf16x32(reinterpret_cast<const __nv_bfloat16*>(e.x) + off, xv);
+        } else {
+          const float4* xp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(e.x) + off);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 a = xp[q];
+            xv[4 * q] = a.x; xv[4 * q + 1] = a.y; xv[4 * q + 2] = a.z; xv[4 * q + 3] = a.w;
+          }
+        }
         const float4* g1 = reinterpret_cast<const float4*>(gt + 32 * c);
         const float4* g2 = reinterpret_cast<const float4*>(gm + 32 * c);
 #pragma unroll
@@ -124,7 +133,14 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
           xv[4 * q + 2] = fmaf(a.z + b.z, v[4 * q + 2], xv[4 * q + 2]);
           xv[4 * q + 3] = fmaf(a.w + b.w, v[4 * q + 3], xv[4 * q + 3]);
         }
-        store_bf16x32(xp, xv);
+        if constexpr (EPI == EPI_RESID) {
+          store_bf16x32(reinterpret_cast<__nv_bfloat16*>(e.x) + off, xv);
+        } else {
+          float4* xp = reinterpret_cast<float4*>(reinterpret_cast<float*>(e.x) + off);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            xp[q] = make_float4(xv[4 * q], xv[4 * q + 1], xv[4 * q + 2], xv[4 * q + 3]);
+        }
       }
     }
   } else if constexpr (EPI == EPI_QKV) {
@@ -339,6 +355,7 @@ cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void*
     case EPI_QKV: return run<EPI_QKV>(M, N, K, A, Bm, e, st);
     case EPI_RESID: return run<EPI_RESID>(M, N, K, A, Bm, e, st);
     case EPI_SWIGLU: return run<EPI_SWIGLU>(M, N, K, A, Bm, e, st);
+    case EPI_RESID_F32: return run<EPI_RESID_F32>(M, N, K, A, Bm, e, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -73,16 +73,23 @@ cudaError_t launch_unpack(const h3_layout* L, int B, int row_elems, const void* 
 // dst[b, perm[j]] = src[b, j] (gather == false, src [B, n, E], dst [B, S_dst, E])
 cudaError_t launch_permute_rows(int B, int n, int S_full, int row_elems, const int32_t* perm,
                                 const void* src, void* dst, bool gather, cudaStream_t st);
+// Same, converting the rows: gather bf16 -> fp32, scatter fp32 -> bf16 (round to nearest even).
+cudaError_t launch_permute_rows_convert(int B, int n, int S_full, int row_elems,
+                                        const int32_t* perm, const void* src, void* dst,
+                                        bool gather, cudaStream_t st);
 
+// x_f32: the residual stream x is fp32 (inside the stack) instead of bf16.
 cudaError_t launch_norm_modulate(const LayoutView& L, int B, int H, int chunk_shift,
-                                 int chunk_scale, float eps, const void* x, const float* table,
-                                 const float* tmod, void* h, cudaStream_t st);
+                                 int chunk_scale, float eps, const void* x, bool x_f32,
+                                 const float* table, const float* tmod, void* h,
+                                 cudaStream_t st);
 
 cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const float* w_t1,
                             const float* w_t2, const float* w_proj, float* tmod, float* ws,
                             cudaStream_t st);
 
-enum GemmEpilogue { EPI_STORE = 0, EPI_QKV = 1, EPI_RESID = 2, EPI_SWIGLU = 3 };
+// EPI_RESID_F32: gated residual on an fp32 residual stream (inside the stack).
+enum GemmEpilogue { EPI_STORE = 0, EPI_QKV = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_RESID_F32 = 4 };
 
 struct GemmEpiArgs {
   LayoutView L;

@@ -218,6 +218,37 @@ __global__ void k_permute(int B, int n, int S_full, int vec_per_row,
   }
 }
 
+// Row gather / scatter with conversion: gather reads bf16 rows and writes fp32,
+// scatter reads fp32 rows and writes bf16 (round to nearest even).
+__global__ void k_permute_convert(int B, int n, int S_full, int vec8_per_row,
+                                  const int32_t* __restrict__ perm, const void* __restrict__ src,
+                                  void* __restrict__ dst, int gather) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       row < (long long)B * n; row += warps) {
+    const int b = (int)(row / n), j = (int)(row % n);
+    const long long full_row = (long long)b * S_full + perm[j];
+    if (gather) {
+      const uint4* sp = reinterpret_cast<const uint4*>(src) + full_row * vec8_per_row;
+      float4* dp = reinterpret_cast<float4*>(dst) + row * vec8_per_row * 2;
+      for (int v = lane; v < vec8_per_row; v += 32) {
+        const uint4 u = sp[v];
+        dp[2 * v] = make_float4(bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y));
+        dp[2 * v + 1] = make_float4(bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w));
+      }
+    } else {
+      const float4* sp = reinterpret_cast<const float4*>(src) + row * vec8_per_row * 2;
+      uint4* dp = reinterpret_cast<uint4*>(dst) + full_row * vec8_per_row;
+      for (int v = lane; v < vec8_per_row; v += 32) {
+        const float4 a = sp[2 * v], c = sp[2 * v + 1];
+        dp[v] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(c.x, c.y),
+                           pack_bf16x2(c.z, c.w));
+      }
+    }
+  }
+}
+
 int grid_for(long long work, int per_block) {
   long long g = (work + per_block - 1) / per_block;
   const long long cap = (long long)num_sms() * 16;
@@ -292,6 +323,16 @@ cudaError_t launch_permute_rows(int B, int n, int S_full, int row_elems, const i
   if (rows == 0) return cudaSuccess;
   k_permute<<<grid_for(rows, 8), 256, 0, st>>>(B, n, S_full, row_elems / 8, perm,
                                                 (const uint4*)src, (uint4*)dst, gather ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_rows_convert(int B, int n, int S_full, int row_elems,
+                                        const int32_t* perm, const void* src, void* dst,
+                                        bool gather, cudaStream_t st) {
+  const long long rows = (long long)B * n;
+  if (rows == 0) return cudaSuccess;
+  k_permute_convert<<<grid_for(rows, 8), 256, 0, st>>>(B, n, S_full, row_elems / 8, perm, src,
+                                                        dst, gather ? 1 : 0);
   return cudaGetLastError();
 }
 

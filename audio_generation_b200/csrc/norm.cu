@@ -17,32 +17,56 @@ namespace {
 
 constexpr int kMaxVecPerLane = 24;  // hidden <= 24 * 256 = 6144
 
+// Eight consecutive fp32 elements of a row.
+__device__ __forceinline__ void load8(const float* p, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// XT is the storage type of the residual stream x: bf16 for a single block,
+// fp32 inside the stack. A bf16 row is held in registers (84 per lane at
+// hidden 5376); an fp32 row is re-read for the second and third pass.
+template <typename XT>
 __global__ void __launch_bounds__(256) k_norm_modulate(
     int rows, int S, int H, int chunk_shift, int chunk_scale, float eps,
-    const uint4* __restrict__ x, const int32_t* __restrict__ tags,
+    const XT* __restrict__ x, const int32_t* __restrict__ tags,
     const int32_t* __restrict__ t_idx, const float* __restrict__ table,
     const float* __restrict__ tmod, uint4* __restrict__ h) {
+  constexpr bool kHold = sizeof(XT) == 2;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int s = row % S;
-  const int nv = H >> 8;  // 16-byte vectors per lane
-  const uint4* xr = x + (size_t)row * (H >> 3);
+  const int nv = H >> 8;  // 8-element vectors per lane
+  const XT* xr = x + (size_t)row * H;
   uint4* hr = h + (size_t)row * (H >> 3);
   const int tag = tags[s];
   if (tag < 0) {
     for (int i = 0; i < nv; ++i) hr[lane + 32 * i] = make_uint4(0, 0, 0, 0);
     return;
   }
-  uint4 v[kMaxVecPerLane];
+  uint4 held[kHold ? kMaxVecPerLane : 1] = {};
+  auto get8 = [&](int i, float* v) {
+    if constexpr (kHold) {
+      const uint4 u = held[i];
+      v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+      v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+    } else {
+      load8(xr + 8 * (lane + 32 * i), v);
+    }
+  };
   float sum = 0.f;
 #pragma unroll
   for (int i = 0; i < kMaxVecPerLane; ++i) {
     if (i < nv) {
-      v[i] = xr[lane + 32 * i];
-      const uint32_t* u = reinterpret_cast<const uint32_t*>(&v[i]);
+      float v[8];
+      if constexpr (kHold) {
+        held[i] = *reinterpret_cast<const uint4*>(xr + 8 * (lane + 32 * i));
+      }
+      get8(i, v);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) sum += bf16lo(u[k]) + bf16hi(u[k]);
+      for (int k = 0; k < 8; ++k) sum += v[k];
     }
   }
 #pragma unroll
@@ -52,11 +76,12 @@ __global__ void __launch_bounds__(256) k_norm_modulate(
 #pragma unroll
   for (int i = 0; i < kMaxVecPerLane; ++i) {
     if (i < nv) {
-      const uint32_t* u = reinterpret_cast<const uint32_t*>(&v[i]);
+      float v[8];
+      get8(i, v);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float a = bf16lo(u[k]) - mean, b = bf16hi(u[k]) - mean;
-        sq += a * a + b * b;
+      for (int k = 0; k < 8; ++k) {
+        const float a = v[k] - mean;
+        sq += a * a;
       }
     }
   }
@@ -71,14 +96,9 @@ __global__ void __launch_bounds__(256) k_norm_modulate(
 #pragma unroll
   for (int i = 0; i < kMaxVecPerLane; ++i) {
     if (i < nv) {
-      const int e4 = 2 * (lane + 32 * i);  // float4 index of the first of 8 elements
-      const uint32_t* u = reinterpret_cast<const uint32_t*>(&v[i]);
+      const int e4 = 2 * (lane + 32 * i);  // float4 index of the first of the 8 elements
       float xs[8];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        xs[2 * k] = bf16lo(u[k]);
-        xs[2 * k + 1] = bf16hi(u[k]);
-      }
+      get8(i, xs);
       float shv[8], scv[8];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
@@ -105,16 +125,22 @@ __global__ void __launch_bounds__(256) k_norm_modulate(
 }  // namespace
 
 cudaError_t launch_norm_modulate(const LayoutView& L, int B, int H, int chunk_shift,
-                                 int chunk_scale, float eps, const void* x, const float* table,
-                                 const float* tmod, void* h, cudaStream_t st) {
+                                 int chunk_scale, float eps, const void* x, bool x_f32,
+                                 const float* table, const float* tmod, void* h,
+                                 cudaStream_t st) {
   const int rows = B * L.S;
   if (rows == 0) return cudaSuccess;
   if (H % 256 != 0 || H / 256 > kMaxVecPerLane) return cudaErrorInvalidValue;
   const int warps_per_block = 8;
   const int grid = (rows + warps_per_block - 1) / warps_per_block;
-  k_norm_modulate<<<grid, 32 * warps_per_block, 0, st>>>(rows, L.S, H, chunk_shift, chunk_scale,
-                                                          eps, (const uint4*)x, L.tags, L.t_idx,
-                                                          table, tmod, (uint4*)h);
+  if (x_f32)
+    k_norm_modulate<float><<<grid, 32 * warps_per_block, 0, st>>>(
+        rows, L.S, H, chunk_shift, chunk_scale, eps, (const float*)x, L.tags, L.t_idx, table,
+        tmod, (uint4*)h);
+  else
+    k_norm_modulate<__nv_bfloat16><<<grid, 32 * warps_per_block, 0, st>>>(
+        rows, L.S, H, chunk_shift, chunk_scale, eps, (const __nv_bfloat16*)x, L.tags, L.t_idx,
+        table, tmod, (uint4*)h);
   return cudaGetLastError();
 }
 

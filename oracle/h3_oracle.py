@@ -93,11 +93,14 @@ def timestep_sinusoid(t: np.ndarray, freq_dim: int) -> np.ndarray:
 
 def timestep_modulation(t: np.ndarray, w_t1: np.ndarray, w_t2: np.ndarray,
                         w_proj: np.ndarray, freq_dim: int, hidden: int) -> np.ndarray:
-    """tmod[n_t, 6, H] = W_proj . SiLU(W_t2 . SiLU(W_t1 . sinusoid(t)))."""
+    """tmod[n_t, 6, H] = W_proj . SiLU(W_t2 . SiLU(W_t1 . sinusoid(t))).
+
+    Given only the first c*H rows of W_proj, returns the first c chunks [n_t, c, H].
+    """
     s = timestep_sinusoid(t, freq_dim)
     temb = silu(s @ np.asarray(w_t1, F).T) @ np.asarray(w_t2, F).T
     tmod = silu(temb) @ np.asarray(w_proj, F).T
-    return tmod.reshape(-1, 6, hidden)
+    return tmod.reshape(tmod.shape[0], -1, hidden)
 
 
 # --------------------------------------------------------------------------

@@ -1,0 +1,131 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point the
+header declares, and rejects bad arguments before touching the device."""
+
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+from audio_generation_b200 import h3
+from workloads import FULL_DIMS, TINY_DIMS, Dims
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "h3.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"^H3_API\s+[\w\s\*]+?\b(h3_\w+)\s*\(", src, re.M)))
+
+
+def exported_symbols():
+    out = subprocess.run(["nm", "-D", "--defined-only", h3.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    return {l.split()[-1] for l in out.splitlines() if " T " in l}
+
+
+def test_library_exports_every_declared_entry_point():
+    decl = header_functions()
+    assert len(decl) >= 19
+    exp = exported_symbols()
+    missing = [n for n in decl if n not in exp]
+    assert not missing, missing
+    # and the binding wires every one of them
+    assert set(decl) <= set(h3._SIGNATURES)
+
+
+def test_only_declared_entry_points_are_exported():
+    exp = {s for s in exported_symbols() if s.startswith("h3_")}
+    assert exp == set(header_functions())
+
+
+def test_status_strings_and_version():
+    assert h3.h3_abi_version() >= 1
+    for code, word in [(0, "ok"), (-1, "argument"), (-2, "shape"), (-3, "aligned"),
+                       (-4, "layout"), (-5, "workspace"), (-6, "CUDA"), (-7, "timed out")]:
+        assert word in h3.h3_status_string(code)
+    assert "unknown" in h3.h3_status_string(42)
+
+
+def _ws_expected(d, B, S):
+    a = lambda n: (n + 255) // 256 * 256
+    rows = B * S
+    A = d.heads * d.head_dim
+    one = a(rows * A * 2)
+    return (a(rows * d.hidden * 2) + max(3 * one, a(rows * d.ffn * 2)) + a(rows * A * 2)
+            + a(rows * d.hidden * 4))
+
+
+@pytest.mark.parametrize("dims,B,S", [(FULL_DIMS, 1, 8192), (TINY_DIMS, 2, 256),
+                                      (FULL_DIMS, 1, 0), (TINY_DIMS, 3, 333)])
+def test_workspace_size(dims, B, S):
+    assert h3.h3_workspace_size(h3.make_dims(dims), B, S) == _ws_expected(dims, B, S)
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 64), ("hidden", 500), ("heads", 5),
+                                         ("ffn", 1000), ("rope_freq_dim", 8)])
+def test_unsupported_dims_are_rejected_on_the_host(field, value):
+    kw = dict(FULL_DIMS.__dict__)
+    kw[field] = value
+    d = h3.make_dims(Dims(**kw))
+    assert h3.h3_workspace_size(d, 1, 128) == 0
+    out = ctypes.c_void_p()
+    desc = h3.h3_layout_desc(S=0)
+    assert h3.lib().h3_layout_prepare(ctypes.byref(d), ctypes.byref(desc), None,
+                                      ctypes.byref(out)) == h3.H3_ERR_SHAPE
+    assert out.value is None
+
+
+def test_null_arguments_are_rejected_on_the_host():
+    L = h3.lib()
+    d = h3.make_dims(TINY_DIMS)
+    out = ctypes.c_void_p()
+    assert L.h3_layout_prepare(ctypes.byref(d), None, None, ctypes.byref(out)) == h3.H3_ERR_ARG
+    desc = h3.h3_layout_desc(S=-1)
+    assert L.h3_layout_prepare(ctypes.byref(d), ctypes.byref(desc), None,
+                               ctypes.byref(out)) == h3.H3_ERR_ARG
+    desc = h3.h3_layout_desc(S=10, n_t=10)  # null tags / positions
+    assert L.h3_layout_prepare(ctypes.byref(d), ctypes.byref(desc), None,
+                               ctypes.byref(out)) == h3.H3_ERR_ARG
+    w = h3.h3_block_weights()
+    assert L.h3_block_forward(ctypes.byref(d), ctypes.byref(w), None, None, None, 1, None, 0,
+                              None) == h3.H3_ERR_ARG
+    assert L.h3_pack_rows(None, 1, 8, None, None, None, None, None) == h3.H3_ERR_ARG
+    assert L.h3_timestep_modulation(ctypes.byref(d), 4, None, None, None, None, None, None, 0,
+                                    None) == h3.H3_ERR_ARG
+    assert L.h3_timestep_modulation(ctypes.byref(d), 0, None, None, None, None, None, None, 0,
+                                    None) == h3.H3_OK  # nothing to do
+    assert L.h3_layout_error(None) == h3.H3_ERR_ARG
+
+
+def test_binding_raises_typed_errors():
+    with pytest.raises(h3.H3Error) as ei:
+        h3._check(h3.H3_ERR_LAYOUT, "x")
+    assert ei.value.status == h3.H3_ERR_LAYOUT
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(h3, "_lib", None)
+    monkeypatch.setattr(h3, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(ImportError):
+        h3.lib()
+
+
+def _imports(path):
+    out = []
+    for dp, _, fs in os.walk(path):
+        for f in fs:
+            if f.endswith(".py"):
+                with open(os.path.join(dp, f)) as fh:
+                    out += re.findall(r"^\s*(?:from|import)\s+([\w\.]+)", fh.read(), re.M)
+    return out
+
+
+def test_product_never_imports_the_oracle_and_vice_versa():
+    assert not any(m.split(".")[0] == "oracle" for m in _imports(os.path.join(ROOT, "audio_generation_b200")))
+    assert not any(m.split(".")[0] in ("audio_generation_b200",) for m in _imports(os.path.join(ROOT, "oracle")))
+    assert not any(m.split(".")[0] in ("audio_generation_b200", "oracle")
+                   for m in _imports(os.path.join(ROOT, "workloads")))

@@ -1,0 +1,138 @@
+"""The block stack (h3_stack_forward) on the GPU.
+
+The stack gathers the valid rows once into an fp32 residual stream, runs every
+block on it with no mask, and scatters the result back (rounded to bf16 once).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from audio_generation_b200 import h3
+from oracle import h3_oracle as O
+from tests.h3_testlib import (DevLayout, DevWeights, assert_close, dev_bf16, dev_f32, host_bits,
+                              host_f64, rel_l2)
+from tests.test_gpu_block import _sample_rows, _tmod_rows_fn, amplified_weights, gpu_tmod
+from workloads import (FULL_DIMS, TINY_DIMS, Dims, Layout, activations, block_weights,
+                       config_layout, normal_bf16, prologue_weights, random_layout)
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_stack(dl, dws, tmod, x, B):
+    ws_b = h3.h3_workspace_size(dl.dims, B, dl.L.S)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+    h3.h3_stack_forward(dl.dims, [w.c for w in dws], dl.handle, tmod, x, B, ws, ws_b)
+    torch.cuda.synchronize()
+    assert h3.h3_layout_error(dl.handle) == h3.H3_OK
+
+
+def test_stack_config1_50_blocks():
+    dims = TINY_DIMS
+    L = config_layout(1)
+    dl = DevLayout(dims, L)
+    pw = prologue_weights(dims, 1)
+    ws_host = [block_weights(dims, 1, i) for i in range(50)]
+    dws = [DevWeights(w) for w in ws_host]
+    xb = activations(dims, 1, L.S)
+    x = dev_bf16(xb)
+    gpu_stack(dl, dws, gpu_tmod(dims, L.timestep, pw), x, 1)
+    got = host_f64(x)[0]
+    x0 = O.bf16_to_f64(xb[0])
+    tm = O.timestep_modulation(L.timestep, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim, dims.hidden)
+    ref = O.stack_forward(x0[None], lambda i: ws_host[i], 50, L, tm, dims)[0]
+    pad = L.tags < 0
+    assert_close(got, ref, what="50-block stack")
+    # The stack rounds its fp32 stream to bf16 once, at the end; that single
+    # rounding (~0.3 bf16 step rms) is ~12% of this small workload's total update,
+    # so the update is compared with the float64 result rounded at the same point.
+    ref_q = O.round_bf16(ref)
+    assert rel_l2(got[~pad] - x0[~pad], ref_q[~pad] - x0[~pad]) < 0.1
+    np.testing.assert_array_equal(got[pad], x0[pad])
+
+
+@pytest.mark.parametrize("S,seed", [(300, 1), (97, 2)])
+def test_stack_small_amplified(S, seed):
+    dims = Dims(hidden=256, heads=2, head_dim=128, ffn=384, time_embed_dim=64, time_hidden=128)
+    L = random_layout(S, seed, pad_runs=3, max_run=60, n_t=5)
+    dl = DevLayout(dims, L)
+    ws_host = [amplified_weights(dims, 10 * seed + i, std=0.05, table_std=0.2) for i in range(4)]
+    dws = [DevWeights(w) for w in ws_host]
+    g = np.random.default_rng([seed, 71])
+    tm = (g.standard_normal((L.n_t, 6, dims.hidden)) * 0.2).astype(np.float32)
+    B = 2
+    xb = normal_bf16((B, S, dims.hidden), [seed, 72], 1.0)
+    x = dev_bf16(xb)
+    gpu_stack(dl, dws, dev_f32(tm), x, B)
+    got = host_f64(x)
+    pad = L.tags < 0
+    for b in range(B):
+        x0 = O.bf16_to_f64(xb[b])
+        ref = O.stack_forward(x0[None], lambda i: ws_host[i], 4, L, tm, dims)[0]
+        assert np.linalg.norm(ref[~pad] - x0[~pad]) > 0.1 * np.linalg.norm(x0[~pad])
+        assert_close(got[b], ref, what="stack x_out", storage_rounding=True)
+        assert_close(got[b, ~pad] - x0[~pad], ref[~pad] - x0[~pad], what="stack update",
+                     mabs=np.inf)
+        np.testing.assert_array_equal(got[b, pad], x0[pad])
+
+
+def test_stack_config5_first_block_sampled_rows():
+    """One block through the stack path (compaction, fp32 stream) on the
+    config-5 layout with its two timesteps, on sampled rows."""
+    dims = FULL_DIMS
+    L = config_layout(5)
+    dl = DevLayout(dims, L)
+    w = block_weights(dims, 5, 0)
+    pw = prologue_weights(dims, 5)
+    xb = activations(dims, 5, L.S)
+    x = dev_bf16(xb)
+    gpu_stack(dl, [DevWeights(w)], gpu_tmod(dims, L.timestep, pw), x, 1)
+    rows = _sample_rows(L)
+    got = host_f64(x[0, torch.from_numpy(rows).cuda()])
+    x0 = O.bf16_to_f64(xb[0])
+    tm = O.timestep_modulation(L.timestep, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim, dims.hidden)
+    ref = O.block_forward_rows(x0, w, L, lambda ti, c: tm[ti, :c], dims, rows)
+    pad = (L.tags < 0)[rows]
+    assert_close(got, ref, what="cfg5 block 0 x_out")
+    assert_close(got[~pad] - x0[rows][~pad], ref[~pad] - x0[rows][~pad], what="cfg5 update",
+                 mabs=np.inf)
+    np.testing.assert_array_equal(got[pad], x0[rows][pad])
+
+
+def _valid_only_layout(L):
+    keep = L.tags >= 0
+    tags = L.tags[keep]
+    return Layout(tags=tags, pos=L.pos[keep], t_idx=L.t_idx[keep], timestep=L.timestep,
+                  video_idx=np.nonzero(tags == 0)[0].astype(np.int32),
+                  audio_idx=np.nonzero(tags == 2)[0].astype(np.int32),
+                  text_idx=np.nonzero(tags == 1)[0].astype(np.int32))
+
+
+def test_stack_config5_50_blocks_properties():
+    """The full 50-block, 16384-row stack: padding rows untouched bit for bit,
+    finite outputs, deterministic, and identical (bit for bit) to the same stack
+    run on the valid rows alone as a padding-free sequence."""
+    dims = FULL_DIMS
+    L = config_layout(5)
+    dl = DevLayout(dims, L)
+    pw = prologue_weights(dims, 5)
+    dws = [DevWeights(block_weights(dims, 5, i)) for i in range(50)]
+    tmod = gpu_tmod(dims, L.timestep, pw)
+    xb = activations(dims, 5, L.S)
+    x1 = dev_bf16(xb)
+    gpu_stack(dl, dws, tmod, x1, 1)
+    out1 = host_bits(x1)[0]
+    pad = L.tags < 0
+    np.testing.assert_array_equal(out1[pad], xb[0, pad])
+    assert np.all(np.isfinite(O.bf16_to_f64(out1)))
+    x2 = dev_bf16(xb)
+    gpu_stack(dl, dws, tmod, x2, 1)
+    np.testing.assert_array_equal(host_bits(x2)[0], out1)
+    Lv = _valid_only_layout(L)
+    dlv = DevLayout(dims, Lv)
+    xv = dev_bf16(np.ascontiguousarray(xb[:, ~pad]))
+    gpu_stack(dlv, dws, tmod, xv, 1)
+    np.testing.assert_array_equal(host_bits(xv)[0], out1[~pad])
+    # the stack moved the valid rows well beyond bf16 resolution
+    d = O.bf16_to_f64(out1[~pad]) - O.bf16_to_f64(xb[0, ~pad])
+    assert np.linalg.norm(d) > 0.5 * np.linalg.norm(O.bf16_to_f64(xb[0, ~pad]))

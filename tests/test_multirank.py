@@ -1,0 +1,61 @@
+"""The benchmark's multi-process plumbing on CPU: two gloo ranks, each timing
+its own replica; the reported time is the maximum over ranks."""
+
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    ws, r, local = bench.dist_env()
+    bench.barrier(ws)
+    t = bench.max_over_ranks(10.0 + 5.0 * rank, ws)
+    bench.barrier(ws)
+    q.put((r, ws, local, t))
+    dist.destroy_process_group()
+
+
+def test_two_ranks_report_the_max_time():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == [(0, 2, 0, 15.0), (1, 2, 1, 15.0)]
+
+
+def test_single_process_defaults():
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        os.environ.pop(k, None)
+    assert bench.dist_env() == (1, 0, 0)
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_work_counts_match_the_stated_flops():
+    from workloads import FULL_DIMS
+    # per-row GEMM flops 770.7 M plus 4 * 56 * 128 flops per (query, key) pair
+    f = bench.block_flops(FULL_DIMS, 8192)
+    assert abs(f - (2 * 8192 * (5376 * 21504 + 7168 * 5376 + 5376 * 28672 + 14336 * 5376)
+                    + 4 * 56 * 128 * 8192 ** 2)) < 1
+    assert abs(f / 1e12 - 8.238) < 0.01
