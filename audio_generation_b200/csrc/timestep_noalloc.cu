@@ -1,0 +1,85 @@
+// h3_timestep_modulation_noalloc: the timestep-modulation prologue for callers
+// that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc (or hand the library a scratch buffer)
+// at the point where they compute the per-forward modulation: a serving loop
+// whose device memory is reserved up front by its own pool and that forbids
+// further device allocations, or a latency-critical loop (an audio/video frame
+// callback) in which allocation is not allowed. This entry point computes the
+// same result as h3_timestep_modulation with its scratch (sinusoid, MLP hidden
+// and time-embedding rows) in a fixed, statically sized device array that
+// belongs to the library; the caller passes only inputs and outputs.
+//
+// Limits and sharing:
+//  - The array holds kStaticScratchBytes (4 MiB); n_t is accepted only while
+//    h3_timestep_workspace_size(dims, n_t) fits in it (at the full constructor
+//    widths, n_t <= 126). Larger requests return H3_ERR_WORKSPACE before any
+//    work is queued.
+//  - Every GPU that loads the library holds its own copy of the array until the
+//    process exits.
+//  - All calls on a device share that one array, and the array keeps the last
+//    call's contents. Nothing in it needs to start at zero (every scratch value
+//    is written before it is read), but calls whose work overlaps on the GPU
+//    (different streams without ordering between them) race on it: order them
+//    on one stream or with events.
+//  - The first call on a device looks up the array's device address
+//    (cudaGetSymbolAddress, with that device current); make that first call
+//    before any stream capture.
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = 4u << 20;
+constexpr int kMaxDevices = 64;
+
+// File-scope device scratch. In host code this name is only a stand-in for the
+// symbol, never a usable address: kernels receive the device address obtained
+// from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_timestep_scratch[kStaticScratchBytes];
+
+std::mutex g_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up once per device).
+h3_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return H3_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return H3_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_timestep_scratch);
+    if (e != cudaSuccess || p == nullptr) return H3_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return H3_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" h3_status h3_timestep_modulation_noalloc(const h3_dims* dims, int n_t, const float* t,
+                                                    const float* w_t1, const float* w_t2,
+                                                    const float* w_proj, float* tmod,
+                                                    h3_stream_t stream) {
+  const size_t need = h3_timestep_workspace_size(dims, n_t);
+  if (dims == nullptr || n_t < 0) return H3_ERR_ARG;
+  if (need == 0 && n_t > 0) return H3_ERR_SHAPE;
+  if (need > kStaticScratchBytes) return H3_ERR_WORKSPACE;
+  if (n_t == 0) return H3_OK;
+  if (!t || !w_t1 || !w_t2 || !w_proj || !tmod) return H3_ERR_ARG;
+  if (!aligned16(t) || !aligned16(w_t1) || !aligned16(w_t2) || !aligned16(w_proj) ||
+      !aligned16(tmod))
+    return H3_ERR_ALIGN;
+  void* scratch = nullptr;
+  const h3_status s = scratch_address(&scratch);
+  if (s != H3_OK) return s;
+  const cudaError_t e = h3::launch_timestep(*dims, n_t, t, w_t1, w_t2, w_proj, tmod,
+                                            static_cast<float*>(scratch),
+                                            reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? H3_OK : H3_ERR_CUDA;
+}

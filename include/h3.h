@@ -181,6 +181,23 @@ H3_API h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const floa
                                  const float* w_t2, const float* w_proj, float* tmod, void* ws,
                                  size_t ws_bytes, h3_stream_t stream);
 
+/* Same result as h3_timestep_modulation, for callers that cannot allocate device
+ * memory (a serving loop whose device memory is reserved up front by its own
+ * pool, or a latency-critical frame callback where allocation is forbidden).
+ * The pages have no counterpart to this entry point; it exists for those
+ * callers. It allocates nothing: its scratch is a fixed 4 MiB device array
+ * inside the library (one per GPU that loads the library, held until exit).
+ * n_t is accepted while h3_timestep_workspace_size(dims, n_t) <= 4 MiB (n_t <= 126
+ * at the full constructor widths); larger n_t returns H3_ERR_WORKSPACE before any
+ * work is queued. All calls on a device share the array: calls whose work
+ * overlaps on the GPU race (order them on one stream or with events). Nothing in
+ * the array needs to start at zero. The first call on a device looks up the
+ * array's address; make it before any stream capture. */
+H3_API h3_status h3_timestep_modulation_noalloc(const h3_dims* dims, int n_t, const float* t,
+                                                const float* w_t1, const float* w_t2,
+                                                const float* w_proj, float* tmod,
+                                                h3_stream_t stream);
+
 /* ---- single steps of the block (each also runs inside h3_block_forward) ---- */
 
 /* a3 / a7 — h = LayerNorm(x) * (1 + scale) + shift (no affine, biased
