@@ -198,10 +198,22 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
   }
 }
 
+// Tile order: the N tiles are cut into groups of `group_n` columns; within a
+// group the tiles run N-fastest, then down M. The CTAs in flight then share a
+// group of weight tiles that stays in L2 while the row blocks stream past it.
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int group_n,
+                                            int& m0, int& n0) {
+  const int per_group = group_n * tiles_m;
+  const int g = t / per_group, r = t - g * per_group;
+  const int width = min(group_n, tiles_n - g * group_n);
+  m0 = (r / width) * BM;
+  n0 = (g * group_n + r % width) * BN;
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           int M, int N, int K, const GemmEpiArgs e) {
+           int M, int N, int K, int group_n, const GemmEpiArgs e) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -249,7 +261,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t n = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
-        const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+        int m0, n0;
+        tile_coords(t, tiles_m, tiles_n, group_n, m0, n0);
         for (int kb = 0; kb < kb_n; ++kb) {
           const uint32_t s = n % STAGES, ph = (n / STAGES) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, wc)) {
@@ -309,7 +322,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t acc = it & 1, aph = (it >> 1) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph, wc))) break;
       tc_fence_after();
-      const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+      int m0, n0;
+      tile_coords(t, tiles_m, tiles_n, group_n, m0, n0);
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       epilogue_tile<EPI>(taddr, m0 + row_local, n0, M, N, e);
       tc_fence_before();
@@ -340,7 +354,12 @@ cudaError_t run(int M, int N, int K, const void* A, const void* Bm, const GemmEp
     return cudaErrorInvalidValue;
   const int T = ((M + BM - 1) / BM) * (N / BN);
   const int grid = T < num_sms() ? T : num_sms();
-  k_gemm<EPI><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, M, N, K, e);
+  // Weight tiles kept L2-resident per group: about 48 MB of B.
+  const long long b_tile_bytes = (long long)BN * K * 2;
+  int group_n = (int)((48ll << 20) / b_tile_bytes);
+  if (group_n < 1) group_n = 1;
+  if (group_n > N / BN) group_n = N / BN;
+  k_gemm<EPI><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, M, N, K, group_n, e);
   return cudaGetLastError();
 }
 
