@@ -1,16 +1,24 @@
 // a4 / a6 / a8 / a9: persistent tcgen05 GEMM, C = A . B^T (bf16 in, fp32 in
 // TMEM), with the block's fused epilogues.
 //
-// Structure (one CTA per SM, 6 warps):
-//   warp 0        TMA producer: 128x64 A and 256x64 B tiles (128-B swizzle)
-//                 into a 4-stage shared-memory ring
-//   warp 1        TMEM owner and MMA issuer: tcgen05.mma M=128 N=256 K=16,
+// Two CTAs of a (2, 1, 1) cluster compute each 256 x 256 output tile together
+// with cta_group::2 MMAs (M = 256, N = 256, K = 16) issued by rank 0: each CTA
+// loads its own 128 rows of A and its own 128-row half of the B tile, and holds
+// its 128 rows of the accumulator in its own TMEM. An MMA instruction costs
+// tens of cycles to issue whatever its size, so the pair form (twice the work
+// of a 128 x 256 MMA per instruction) keeps the tensor core fed; it also
+// halves each SM's share of B traffic and shared-memory operand reads.
+// Per CTA (6 warps):
+//   warp 0        TMA producer: 128x64 A and 128x64 B-half tiles (128-B
+//                 swizzle) into a 6-stage shared-memory ring; completion is
+//                 counted on rank 0's barrier for both CTAs
+//   warp 1        TMEM owner (both CTAs) and, in rank 0, the MMA issuer;
 //                 accumulator double-buffered in TMEM (2 x 256 columns)
-//   warps 2..5    epilogue: tcgen05.ld of the accumulator (one TMEM lane per
-//                 row), fused math, global stores; overlaps the next tile's
-//                 main loop
-// Tiles are walked M-fastest so that the CTAs in flight share B (weights)
-// tiles and re-read A (activations) from L2.
+//   warps 2..5    epilogue: tcgen05.ld of the CTA's 128 accumulator rows (one
+//                 TMEM lane per row), fused math, global stores; overlaps the
+//                 next tile's main loop
+// Tiles run in N-groups whose weight tiles stay L2-resident while the row
+// blocks stream past them.
 //
 // Epilogues:
 //   EPI_QKV    head-interleaved QKV rows ("MiniMax H3 Inference Engine voor Mac
@@ -32,13 +40,10 @@
 namespace h3 {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;  // BM: rows per CTA; a pair tile is 2 BM x BN
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
-constexpr int B_STAGE = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 192;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
 __device__ __forceinline__ void store_bf16x32(void* dst, const float* y) {
   uint4* d = reinterpret_cast<uint4*>(dst);
@@ -210,33 +215,40 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
   n0 = (g * group_n + r % width) * BN;
 }
 
+constexpr int PNST = 6;
+constexpr int P_STAGE = 2 * BM * BK * 2;  // A rows + B half: 32 KB
+constexpr int P_SMEM_BYTES = PNST * P_STAGE + 1024 + 256;
+
 template <int EPI>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           int M, int N, int K, int group_n, const GemmEpiArgs e) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                int M, int N, int K, int group_n, const GemmEpiArgs e) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + PNST * P_STAGE);
+  uint64_t* empty = full + PNST;
+  uint64_t* tfull = empty + PNST;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_m = (M + BM - 1) / BM, tiles_n = N / BN;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int tiles_m = (M + 2 * BM - 1) / (2 * BM), tiles_n = N / BN;
   const int T = tiles_m * tiles_n, kb_n = K / BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < PNST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -247,119 +259,129 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers and TMEM exist before either uses the other's
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{e.L.err, abort_flag};
+  auto at = [&](uint64_t* bar, uint32_t r) { return mapa_shared(smem_u32(bar), r); };
 
   if (warp == 0) {
     if (lane == 0) {
       uint32_t n = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+      for (int t = pair; t < T && ok; t += n_pairs) {
         int m0, n0;
         tile_coords(t, tiles_m, tiles_n, group_n, m0, n0);
+        m0 = 2 * m0 + BM * rank;  // tile_coords counts 128-row units; pair tiles are 256 rows
         for (int kb = 0; kb < kb_n; ++kb) {
-          const uint32_t s = n % STAGES, ph = (n / STAGES) & 1;
+          const uint32_t s = n % PNST, ph = (n / PNST) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, wc)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + s * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_2d(sa, &tmA, &full[s], kb * BK, m0);
-          tma_load_2d(sa + A_STAGE, &tmB, &full[s], kb * BK, n0);
+          uint8_t* sa = smem + s * P_STAGE;
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE);
+          tma_load_2d_pair(sa, &tmA, at(&full[s], 0), kb * BK, m0);
+          tma_load_2d_pair(sa + A_STAGE, &tmB, at(&full[s], 0), kb * BK, n0 + BM * rank);
           ++n;
         }
       }
-      if (!ok) {  // let issued copies land before the CTA retires
-        const uint32_t first = n > STAGES ? n - STAGES : 0;
-        for (uint32_t i = first; i < n; ++i) mbar_drain(&full[i % STAGES], (i / STAGES) & 1);
+      if (!ok && leader) {  // let issued copies land before the CTA retires
+        const uint32_t first = n > PNST ? n - PNST : 0;
+        for (uint32_t i = first; i < n; ++i) mbar_drain(&full[i % PNST], (i / PNST) & 1);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, false, false);
+      constexpr uint32_t hi = sdesc_hi_sw128(1024);
+      const uint32_t base_lo = sdesc_lo(smem_u32(smem), 16);
       uint32_t n = 0, it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < T && ok; t += gridDim.x, ++it) {
+      for (int t = pair; t < T && ok; t += n_pairs, ++it) {
         const uint32_t acc = it & 1, aph = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], aph ^ 1, wc)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
         for (int kb = 0; kb < kb_n; ++kb) {
-          const uint32_t s = n % STAGES, ph = (n / STAGES) & 1;
+          const uint32_t s = n % PNST, ph = (n / PNST) & 1;
           if (!mbar_wait(&full[s], ph, wc)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
-          const uint32_t b0 = a0 + A_STAGE;
+          const uint32_t a_lo = base_lo + s * (P_STAGE >> 4);
+          const uint32_t b_lo = a_lo + (A_STAGE >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            umma_bf16_ss(d, sdesc_sw128(a0 + 32 * k, 16, 1024), sdesc_sw128(b0 + 32 * k, 16, 1024),
-                         idesc, (kb | k) != 0 ? 1u : 0u);
-          }
-          umma_commit(&empty[s]);
+          for (int k = 0; k < BK / 16; ++k)
+            umma_ss_w_pair(d, a_lo + 2 * k, hi, b_lo + 2 * k, hi, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair(at(&empty[s], 0));
+          umma_commit_pair(at(&empty[s], 1));
           ++n;
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        umma_commit_pair(at(&tfull[acc], 0));
+        umma_commit_pair(at(&tfull[acc], 1));
       }
-      umma_commit(drain);  // every MMA this thread issued is complete past this point
+      umma_commit_pair(at(drain, 0));  // every MMA issued is complete past this point
       mbar_drain(drain, 0);
     }
   } else {
     const int quarter = warp & 3;
     const int row_local = quarter * 32 + lane;
+    const uint32_t tempty0 = at(&tempty[0], 0), tempty1 = at(&tempty[1], 0);
     uint32_t it = 0;
-    for (int t = blockIdx.x; t < T; t += gridDim.x, ++it) {
+    for (int t = pair; t < T; t += n_pairs, ++it) {
       const uint32_t acc = it & 1, aph = (it >> 1) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph, wc))) break;
       tc_fence_after();
       int m0, n0;
       tile_coords(t, tiles_m, tiles_n, group_n, m0, n0);
+      m0 = 2 * m0 + BM * rank;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       epilogue_tile<EPI>(taddr, m0 + row_local, n0, M, N, e);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty1 : tempty0);
     }
   }
   __syncthreads();
+  cluster_sync();  // no CTA leaves while the pair's MMAs or signals may still reach it
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
 template <int EPI>
 cudaError_t run(int M, int N, int K, const void* A, const void* Bm, const GemmEpiArgs& e,
                 cudaStream_t st) {
-  cudaError_t err =
-      cudaFuncSetAttribute(k_gemm<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  cudaError_t err = cudaFuncSetAttribute(k_gemm_pair<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         P_SMEM_BYTES);
   if (err != cudaSuccess) return err;
   CUtensorMap ta, tb;
   const uint64_t da[2] = {(uint64_t)K, (uint64_t)M}, sa[1] = {(uint64_t)K * 2};
   const uint32_t ba[2] = {BK, BM};
   const uint64_t db[2] = {(uint64_t)K, (uint64_t)N}, sb[1] = {(uint64_t)K * 2};
-  const uint32_t bb[2] = {BK, BN};
+  const uint32_t bb[2] = {BK, BM};  // each CTA of the pair loads 128 of the tile's 256 B rows
   if (!make_tmap_bf16(&ta, A, 2, da, sa, ba) || !make_tmap_bf16(&tb, Bm, 2, db, sb, bb))
     return cudaErrorInvalidValue;
-  const int T = ((M + BM - 1) / BM) * (N / BN);
-  const int grid = T < num_sms() ? T : num_sms();
+  const int T = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
+  const int max_pairs = num_sms() / 2;
+  const int n_pairs = T < max_pairs ? T : max_pairs;
   // Weight tiles kept L2-resident per group: about 48 MB of B.
   const long long b_tile_bytes = (long long)BN * K * 2;
   int group_n = (int)((48ll << 20) / b_tile_bytes);
   if (group_n < 1) group_n = 1;
   if (group_n > N / BN) group_n = N / BN;
-  k_gemm<EPI><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ta, tb, M, N, K, group_n, e);
+  k_gemm_pair<EPI><<<2 * n_pairs, NUM_THREADS, P_SMEM_BYTES, st>>>(ta, tb, M, N, K, group_n, e);
   return cudaGetLastError();
 }
 

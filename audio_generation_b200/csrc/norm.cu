@@ -7,33 +7,41 @@
 // and pre-feed-forward norms). shift / scale = ada_table[tag] + tmod[t_idx].
 //
 // HBM-bound: per row it reads H bf16 of x, 2H fp32 of tmod (per-row timestep)
-// and writes H bf16 of h; the 3-row AdaLN table stays in L2. All traffic is
-// 16-byte vectors, lane-interleaved so a warp touches 512 contiguous bytes.
+// and writes H bf16 of h; the 3-row AdaLN table stays in L2, and the second
+// read of x hits L1 / L2. All traffic is 16-byte vectors, lane-interleaved so a
+// warp touches 512 contiguous bytes.
 #include "internal.cuh"
 #include "sm100.cuh"
 
 namespace h3 {
 namespace {
 
-constexpr int kMaxVecPerLane = 24;  // hidden <= 24 * 256 = 6144
+constexpr int kMaxVecPerLane = 24;  // hidden <= 24 * 256 = 6144 (a limit of the other kernels)
 
-// Eight consecutive fp32 elements of a row.
+// Eight consecutive elements of a row, as floats.
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* v) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
 __device__ __forceinline__ void load8(const float* p, float* v) {
-  const float4 a = *reinterpret_cast<const float4*>(p);
-  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
 // XT is the storage type of the residual stream x: bf16 for a single block,
-// fp32 inside the stack. A bf16 row is held in registers (84 per lane at
-// hidden 5376); an fp32 row is re-read for the second and third pass.
+// fp32 inside the stack. Pass 1 accumulates the sum and the sum of squares of
+// x - c (c = the row's first element, so the variance keeps its precision when
+// the mean is far from zero); pass 2 reads x again (L1 / L2) together with the
+// row's modulation and writes h. Nothing is held across the passes, so the
+// kernel runs with few registers and many rows in flight per SM.
 template <typename XT>
 __global__ void __launch_bounds__(256) k_norm_modulate(
     int rows, int S, int H, int chunk_shift, int chunk_scale, float eps,
     const XT* __restrict__ x, const int32_t* __restrict__ tags,
     const int32_t* __restrict__ t_idx, const float* __restrict__ table,
     const float* __restrict__ tmod, uint4* __restrict__ h) {
-  constexpr bool kHold = sizeof(XT) == 2;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -46,79 +54,62 @@ __global__ void __launch_bounds__(256) k_norm_modulate(
     for (int i = 0; i < nv; ++i) hr[lane + 32 * i] = make_uint4(0, 0, 0, 0);
     return;
   }
-  uint4 held[kHold ? kMaxVecPerLane : 1] = {};
-  auto get8 = [&](int i, float* v) {
-    if constexpr (kHold) {
-      const uint4 u = held[i];
-      v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-      v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
-    } else {
-      load8(xr + 8 * (lane + 32 * i), v);
-    }
-  };
-  float sum = 0.f;
-#pragma unroll
-  for (int i = 0; i < kMaxVecPerLane; ++i) {
-    if (i < nv) {
-      float v[8];
-      if constexpr (kHold) {
-        held[i] = *reinterpret_cast<const uint4*>(xr + 8 * (lane + 32 * i));
-      }
-      get8(i, v);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) sum += v[k];
-    }
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const float mean = sum / (float)H;
-  float sq = 0.f;
-#pragma unroll
-  for (int i = 0; i < kMaxVecPerLane; ++i) {
-    if (i < nv) {
-      float v[8];
-      get8(i, v);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float a = v[k] - mean;
-        sq += a * a;
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-  const float rstd = rsqrtf(sq / (float)H + eps);
   const int ti = t_idx[s];
+  float c;
+  {
+    float v[8];
+    load8(xr, v);
+    c = __shfl_sync(0xffffffffu, v[0], 0);
+  }
+  float sum = 0.f, sq = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < nv; ++i) {
+    float v[8];
+    load8(xr + 8 * (lane + 32 * i), v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float d = v[k] - c;
+      sum += d;
+      sq = fmaf(d, d, sq);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  }
+  const float dm = sum / (float)H;
+  const float mean = c + dm;
+  const float var = fmaxf(sq / (float)H - dm * dm, 0.f);
+  const float rstd = rsqrtf(var + eps);
   const float4* sh_t = reinterpret_cast<const float4*>(table + ((size_t)tag * 6 + chunk_shift) * H);
   const float4* sc_t = reinterpret_cast<const float4*>(table + ((size_t)tag * 6 + chunk_scale) * H);
   const float4* sh_m = reinterpret_cast<const float4*>(tmod + ((size_t)ti * 6 + chunk_shift) * H);
   const float4* sc_m = reinterpret_cast<const float4*>(tmod + ((size_t)ti * 6 + chunk_scale) * H);
+#pragma unroll 2
+  for (int i = 0; i < nv; ++i) {
+    const int e4 = 2 * (lane + 32 * i);  // float4 index of the first of the 8 elements
+    float xs[8];
+    load8(xr + 8 * (lane + 32 * i), xs);
+    float shv[8], scv[8];
 #pragma unroll
-  for (int i = 0; i < kMaxVecPerLane; ++i) {
-    if (i < nv) {
-      const int e4 = 2 * (lane + 32 * i);  // float4 index of the first of the 8 elements
-      float xs[8];
-      get8(i, xs);
-      float shv[8], scv[8];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const float4 a = __ldg(sh_t + e4 + q), b = __ldg(sh_m + e4 + q);
-        const float4 c = __ldg(sc_t + e4 + q), d = __ldg(sc_m + e4 + q);
-        shv[4 * q + 0] = a.x + b.x; shv[4 * q + 1] = a.y + b.y;
-        shv[4 * q + 2] = a.z + b.z; shv[4 * q + 3] = a.w + b.w;
-        scv[4 * q + 0] = c.x + d.x; scv[4 * q + 1] = c.y + d.y;
-        scv[4 * q + 2] = c.z + d.z; scv[4 * q + 3] = c.w + d.w;
-      }
-      uint4 out;
-      uint32_t* o = reinterpret_cast<uint32_t*>(&out);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float y0 = (xs[2 * k] - mean) * rstd * (1.f + scv[2 * k]) + shv[2 * k];
-        const float y1 = (xs[2 * k + 1] - mean) * rstd * (1.f + scv[2 * k + 1]) + shv[2 * k + 1];
-        o[k] = pack_bf16x2(y0, y1);
-      }
-      hr[lane + 32 * i] = out;
+    for (int q = 0; q < 2; ++q) {
+      const float4 a = __ldg(sh_t + e4 + q), b = __ldg(sh_m + e4 + q);
+      const float4 cc = __ldg(sc_t + e4 + q), d = __ldg(sc_m + e4 + q);
+      shv[4 * q + 0] = a.x + b.x; shv[4 * q + 1] = a.y + b.y;
+      shv[4 * q + 2] = a.z + b.z; shv[4 * q + 3] = a.w + b.w;
+      scv[4 * q + 0] = cc.x + d.x; scv[4 * q + 1] = cc.y + d.y;
+      scv[4 * q + 2] = cc.z + d.z; scv[4 * q + 3] = cc.w + d.w;
     }
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float y0 = (xs[2 * k] - mean) * rstd * (1.f + scv[2 * k]) + shv[2 * k];
+      const float y1 = (xs[2 * k + 1] - mean) * rstd * (1.f + scv[2 * k + 1]) + shv[2 * k + 1];
+      o[k] = pack_bf16x2(y0, y1);
+    }
+    hr[lane + 32 * i] = out;
   }
 }
 
