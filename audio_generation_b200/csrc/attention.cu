@@ -9,7 +9,8 @@
 //   warps 0..3   softmax of query tile 0 (one row per thread = one TMEM lane)
 //   warps 4..7   softmax of query tile 1
 //   warp 8       TMA producer: both Q tiles once, K and V tiles double-buffered
-//   warp 9       TMEM owner and MMA issuer
+//   warp 9       TMEM owner and MMA issuer (the whole warp runs the issue loop;
+//                one elected lane issues each tcgen05 instruction)
 //   warps 10, 11 idle (they complete the third warpgroup, whose register
 //                budget is handed to the softmax warpgroups)
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512). A
@@ -226,11 +227,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp runs the loop; one lane elected per instruction issues
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
       const uint32_t q_s = smem_u32(smem + OFF_Q);
-      bool ok = mbar_wait(&bars->q_full, 0, wc);
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
+      };
+      bool ok = wait_all(&bars->q_full, 0);
       tc_fence_after();
       // S_i(j) = Q_i K_j^T into TMEM columns [128 i, 128 i + 128)
       constexpr uint32_t hi = sdesc_hi_sw128(1024);
@@ -240,7 +244,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto issue_s = [&](int i, int j) -> bool {
         const int st = j & 1;
         if (i == 0) {
-          if (!mbar_wait(&bars->k_full[st], (j >> 1) & 1, wc)) return false;
+          if (!wait_all(&bars->k_full[st], (j >> 1) & 1)) return false;
           tc_fence_after();
         }
         const uint32_t kl = k_lo + st * (TILE_BYTES >> 4);
@@ -248,26 +252,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
-          umma_ss_w(tmem + i * 128, ql + off, hi, kl + off, hi, idesc_s, kk > 0 ? 1u : 0u);
+          umma_ss_w_elect(tmem + i * 128, ql + off, hi, kl + off, hi, idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->s_full[i]);
-        if (i == 1) umma_commit(&bars->k_empty[st]);
+        umma_commit_elect(&bars->s_full[i]);
+        if (i == 1) umma_commit_elect(&bars->k_empty[st]);
         return true;
       };
       // O_i += P_i(j) V_j, P_i from TMEM columns [128 i, 128 i + 64)
       auto issue_pv = [&](int i, int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(&bars->p_full[i], j & 1, wc)) return false;
-        if (i == 0 && !mbar_wait(&bars->v_full[st], (j >> 1) & 1, wc)) return false;
+        if (!wait_all(&bars->p_full[i], j & 1)) return false;
+        if (i == 0 && !wait_all(&bars->v_full[st], (j >> 1) & 1)) return false;
         tc_fence_after();
         const uint32_t vl = v_lo + st * (TILE_BYTES >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          umma_ts_w(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, vl + kk * (2048 >> 4), hi,
-                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_w_elect(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, vl + kk * (2048 >> 4), hi,
+                          idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        if (i == 1) umma_commit(&bars->v_empty[st]);
-        if (j == n - 1) umma_commit(&bars->o_final[i]);
+        if (i == 1) umma_commit_elect(&bars->v_empty[st]);
+        if (j == n - 1) umma_commit_elect(&bars->o_final[i]);
         return true;
       };
       if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (ok) ok = issue_pv(1, j);
         if (ok && j + 1 < n) ok = issue_s(1, j + 1);
       }
-      umma_commit(&bars->drain);  // every MMA this thread issued is complete past this point
+      umma_commit_elect(&bars->drain);  // every MMA issued is complete past this point
       mbar_drain(&bars->drain, 0);
     }
   }

@@ -216,8 +216,11 @@ H3_API h3_status h3_qkv_rope(const h3_dims* dims, h3_layout_t layout, int B, con
                       void* k, void* v, h3_stream_t stream);
 
 /* a5 — o = softmax(q k^T / sqrt(D)) v per head over the row's document
- * (valid rows attend valid rows; padding query rows are not computed and
- * their output rows are zero). q, k, v [B, NH, S, D] bf16 -> o [B, S, NH*D] bf16. */
+ * (valid rows attend valid rows). Output rows of padding queries carry no
+ * result: rows of 128-row tiles that hold only padding are written as zeros;
+ * padding rows inside mixed tiles hold finite values that every later step
+ * ignores (they are never read back into x). q, k, v [B, NH, S, D] bf16 ->
+ * o [B, S, NH*D] bf16. */
 H3_API h3_status h3_attention(const h3_dims* dims, h3_layout_t layout, int B, const void* q,
                        const void* k, const void* v, void* o, h3_stream_t stream);
 

@@ -23,6 +23,7 @@ CASES = {
     "tiny_cfg1_B2": (TINY_DIMS, lambda: config_layout(1), 2),
     "tiny_rand333": (TINY_DIMS, lambda: random_layout(333, 5, pad_runs=3, max_run=70), 1),
     "full_rand300": (FULL_DIMS, lambda: random_layout(300, 6, pad_runs=2, max_run=50), 1),
+    "tiny_rand1500": (TINY_DIMS, lambda: random_layout(1500, 7, pad_runs=4, max_run=300), 1),
 }
 
 
@@ -85,7 +86,8 @@ def _attention_inputs(dims, L, B, seed, q_scale=1.0):
 
 
 @pytest.mark.parametrize("case,q_scale", [("tiny_cfg1_B2", 1.0), ("tiny_rand333", 1.0),
-                                          ("tiny_rand333", 6.0), ("full_rand300", 1.0)])
+                                          ("tiny_rand333", 6.0), ("full_rand300", 1.0),
+                                          ("tiny_rand1500", 1.0), ("tiny_rand1500", 6.0)])
 def test_attention(case, q_scale):
     dims, L, dl, w, B = _setup(case)
     NH, D = dims.heads, dims.head_dim
