@@ -12,7 +12,8 @@
 //   warp 0        TMA producer: 128x64 A and 128x64 B-half tiles (128-B
 //                 swizzle) into a 6-stage shared-memory ring; completion is
 //                 counted on rank 0's barrier for both CTAs
-//   warp 1        TMEM owner (both CTAs) and, in rank 0, the MMA issuer;
+//   warp 1        TMEM owner (both CTAs) and, in rank 0, the MMA issuer (the
+//                 whole warp runs the loop, an elected lane issues);
 //                 accumulator double-buffered in TMEM (2 x 256 columns)
 //   warps 2..5    epilogue: tcgen05.ld of the CTA's 128 accumulator rows (one
 //                 TMEM lane per row), fused math, global stores; overlaps the
@@ -297,7 +298,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
+    if (leader) {  // the whole warp runs the loop; one elected lane issues
       constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, false, false);
       constexpr uint32_t hi = sdesc_hi_sw128(1024);
       const uint32_t base_lo = sdesc_lo(smem_u32(smem), 16);
@@ -305,12 +306,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int t = pair; t < T && ok; t += n_pairs, ++it) {
         const uint32_t acc = it & 1, aph = (it >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], aph ^ 1, wc)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], aph ^ 1, wc))) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
         for (int kb = 0; kb < kb_n; ++kb) {
           const uint32_t s = n % PNST, ph = (n / PNST) & 1;
-          if (!mbar_wait(&full[s], ph, wc)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, wc))) {
             ok = false;
             break;
           }
@@ -319,16 +320,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b_lo = a_lo + (A_STAGE >> 4);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_ss_w_pair(d, a_lo + 2 * k, hi, b_lo + 2 * k, hi, idesc, (kb | k) != 0 ? 1u : 0u);
-          umma_commit_pair(at(&empty[s], 0));
-          umma_commit_pair(at(&empty[s], 1));
+            umma_ss_w_pair_elect(d, a_lo + 2 * k, hi, b_lo + 2 * k, hi, idesc,
+                                 (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair_elect(at(&empty[s], 0));
+          umma_commit_pair_elect(at(&empty[s], 1));
           ++n;
         }
         if (!ok) break;
-        umma_commit_pair(at(&tfull[acc], 0));
-        umma_commit_pair(at(&tfull[acc], 1));
+        umma_commit_pair_elect(at(&tfull[acc], 0));
+        umma_commit_pair_elect(at(&tfull[acc], 1));
       }
-      umma_commit_pair(at(drain, 0));  // every MMA issued is complete past this point
+      umma_commit_pair_elect(at(drain, 0));  // every MMA issued is complete past this point
       mbar_drain(drain, 0);
     }
   } else {
