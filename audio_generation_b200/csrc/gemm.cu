@@ -1,20 +1,22 @@
 // a4 / a6 / a8 / a9: persistent tcgen05 GEMM, C = A . B^T (bf16 in, fp32 in
 // TMEM), with the block's fused epilogues.
 //
-// Two CTAs of a (2, 1, 1) cluster compute each 256 x 256 output tile together
-// with cta_group::2 MMAs (M = 256, N = 256, K = 16) issued by rank 0: each CTA
-// loads its own 128 rows of A and its own 128-row half of the B tile, and holds
-// its 128 rows of the accumulator in its own TMEM. An MMA instruction costs
-// tens of cycles to issue whatever its size, so the pair form (twice the work
-// of a 128 x 256 MMA per instruction) keeps the tensor core fed; it also
+// Two CTAs of a (2, 1, 1) cluster compute each 256 x BN output tile together
+// with cta_group::2 MMAs (M = 256, N = BN, K = 16) issued by rank 0: each CTA
+// loads its own 128 rows of A and its own BN / 2-row half of the B tile, and
+// holds its 128 rows of the accumulator in its own TMEM. An MMA instruction
+// costs tens of cycles to issue whatever its size, so the pair form (twice the
+// work of a 128-row MMA per instruction) keeps the tensor core fed; it also
 // halves each SM's share of B traffic and shared-memory operand reads.
+// BN is 256, or 224 for the gated-residual GEMMs when that fills the last wave
+// of tiles better (the launcher compares waves x tile width for both).
 // Per CTA (6 warps):
-//   warp 0        TMA producer: 128x64 A and 128x64 B-half tiles (128-B
+//   warp 0        TMA producer: 128x64 A and (BN/2)x64 B-half tiles (128-B
 //                 swizzle) into a 6-stage shared-memory ring; completion is
 //                 counted on rank 0's barrier for both CTAs
 //   warp 1        TMEM owner (both CTAs) and, in rank 0, the MMA issuer (the
 //                 whole warp runs the loop, an elected lane issues);
-//                 accumulator double-buffered in TMEM (2 x 256 columns)
+//                 accumulator double-buffered in TMEM (2 x BN columns)
 //   warps 2..5    epilogue: tcgen05.ld of the CTA's 128 accumulator rows (one
 //                 TMEM lane per row), fused math, global stores; overlaps the
 //                 next tile's main loop
@@ -41,7 +43,10 @@
 namespace h3 {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64;  // BM: rows per CTA; a pair tile is 2 BM x BN
+constexpr int BM = 128, BK = 64;  // BM: rows per CTA; a pair tile is 2 BM x BN
+// Tile width BN: 256, or 224 for the gated-residual GEMMs whose N is a
+// multiple of 224 (N = 5376 gives 24 tiles of 224 instead of 21 of 256, so the
+// 768 tiles fill the 74 CTA pairs' last wave better than 672 do).
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 192;
@@ -81,14 +86,14 @@ __device__ __forceinline__ void ld_acc(uint32_t taddr, float* v) {
 
 // Epilogue for one 128 x 256 accumulator tile. Every lane of the warp executes
 // the TMEM loads (they are warp-collective); stores are predicated per row.
-template <int EPI>
+template <int EPI, int BN>
 __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int M, int N,
                                               const GemmEpiArgs& e) {
   const bool row_ok = m < M;
   if constexpr (EPI == EPI_STORE) {
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out);
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < BN / 32; ++c) {
       float v[32];
       ld_acc(taddr + 32 * c, v);
       if (row_ok) store_bf16x32(out + (size_t)m * N + n0 + 32 * c, v);
@@ -113,7 +118,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
     const float* gt = e.table + ((size_t)(active ? tag : 0) * 6 + e.gate_chunk) * N + n0;
     const float* gm = e.tmod + ((size_t)ti * 6 + e.gate_chunk) * N + n0;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < BN / 32; ++c) {
       float v[32];
       ld_acc(taddr + 32 * c, v);
       if (active) {
@@ -207,6 +212,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
 // Tile order: the N tiles are cut into groups of `group_n` columns; within a
 // group the tiles run N-fastest, then down M. The CTAs in flight then share a
 // group of weight tiles that stays in L2 while the row blocks stream past it.
+template <int BN>
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int group_n,
                                             int& m0, int& n0) {
   const int per_group = group_n * tiles_m;
@@ -217,16 +223,21 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 }
 
 constexpr int PNST = 6;
-constexpr int P_STAGE = 2 * BM * BK * 2;  // A rows + B half: 32 KB
-constexpr int P_SMEM_BYTES = PNST * P_STAGE + 1024 + 256;
+// Stage: 128 A rows + the CTA's BN / 2 B rows, 64 K-elements each (multiple of 1 KB).
+template <int BN>
+constexpr int p_stage() { return (BM + BN / 2) * BK * 2; }
+template <int BN>
+constexpr int p_smem_bytes() { return PNST * p_stage<BN>() + 1024 + 256; }
 
-template <int EPI>
+template <int EPI, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 int M, int N, int K, int group_n, const GemmEpiArgs e) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int P_STAGE = p_stage<BN>();
+  static_assert(P_STAGE % 1024 == 0, "stage alignment");
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + PNST * P_STAGE);
   uint64_t* empty = full + PNST;
   uint64_t* tfull = empty + PNST;
@@ -277,7 +288,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int t = pair; t < T && ok; t += n_pairs) {
         int m0, n0;
-        tile_coords(t, tiles_m, tiles_n, group_n, m0, n0);
+        tile_coords<BN>(t, tiles_m, tiles_n, group_n, m0, n0);
         m0 = 2 * m0 + BM * rank;  // tile_coords counts 128-row units; pair tiles are 256 rows
         for (int kb = 0; kb < kb_n; ++kb) {
           const uint32_t s = n % PNST, ph = (n / PNST) & 1;
@@ -288,7 +299,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           uint8_t* sa = smem + s * P_STAGE;
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE);
           tma_load_2d_pair(sa, &tmA, at(&full[s], 0), kb * BK, m0);
-          tma_load_2d_pair(sa + A_STAGE, &tmB, at(&full[s], 0), kb * BK, n0 + BM * rank);
+          tma_load_2d_pair(sa + A_STAGE, &tmB, at(&full[s], 0), kb * BK, n0 + (BN / 2) * rank);
           ++n;
         }
       }
@@ -343,10 +354,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph, wc))) break;
       tc_fence_after();
       int m0, n0;
-      tile_coords(t, tiles_m, tiles_n, group_n, m0, n0);
+      tile_coords<BN>(t, tiles_m, tiles_n, group_n, m0, n0);
       m0 = 2 * m0 + BM * rank;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-      epilogue_tile<EPI>(taddr, m0 + row_local, n0, M, N, e);
+      epilogue_tile<EPI, BN>(taddr, m0 + row_local, n0, M, N, e);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty1 : tempty0);
@@ -361,10 +372,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, int BN>
 cudaError_t run(int M, int N, int K, const void* A, const void* Bm, const GemmEpiArgs& e,
                 cudaStream_t st) {
-  cudaError_t err = cudaFuncSetAttribute(k_gemm_pair<EPI>,
+  constexpr int P_SMEM_BYTES = p_smem_bytes<BN>();
+  cudaError_t err = cudaFuncSetAttribute(k_gemm_pair<EPI, BN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          P_SMEM_BYTES);
   if (err != cudaSuccess) return err;
@@ -372,7 +384,7 @@ cudaError_t run(int M, int N, int K, const void* A, const void* Bm, const GemmEp
   const uint64_t da[2] = {(uint64_t)K, (uint64_t)M}, sa[1] = {(uint64_t)K * 2};
   const uint32_t ba[2] = {BK, BM};
   const uint64_t db[2] = {(uint64_t)K, (uint64_t)N}, sb[1] = {(uint64_t)K * 2};
-  const uint32_t bb[2] = {BK, BM};  // each CTA of the pair loads 128 of the tile's 256 B rows
+  const uint32_t bb[2] = {BK, BN / 2};  // each CTA of the pair loads half of the tile's B rows
   if (!make_tmap_bf16(&ta, A, 2, da, sa, ba) || !make_tmap_bf16(&tb, Bm, 2, db, sb, bb))
     return cudaErrorInvalidValue;
   const int T = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
@@ -383,8 +395,16 @@ cudaError_t run(int M, int N, int K, const void* A, const void* Bm, const GemmEp
   int group_n = (int)((48ll << 20) / b_tile_bytes);
   if (group_n < 1) group_n = 1;
   if (group_n > N / BN) group_n = N / BN;
-  k_gemm_pair<EPI><<<2 * n_pairs, NUM_THREADS, P_SMEM_BYTES, st>>>(ta, tb, M, N, K, group_n, e);
+  k_gemm_pair<EPI, BN><<<2 * n_pairs, NUM_THREADS, P_SMEM_BYTES, st>>>(ta, tb, M, N, K, group_n, e);
   return cudaGetLastError();
+}
+
+// Waves x tile width for a tile width: the time of the persistent loop in
+// units of one 256-wide tile column, up to the per-tile constant.
+long long wave_cost(int M, int N, int bn) {
+  const long long tiles = (long long)((M + 2 * BM - 1) / (2 * BM)) * (N / bn);
+  const long long pairs = num_sms() / 2;
+  return (tiles + pairs - 1) / pairs * bn;
 }
 
 }  // namespace
@@ -392,13 +412,20 @@ cudaError_t run(int M, int N, int K, const void* A, const void* Bm, const GemmEp
 cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void* Bm,
                         const GemmEpiArgs& e, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  if (N % BN != 0 || K % BK != 0 || K == 0) return cudaErrorInvalidValue;
+  if (N % 256 != 0 || K % BK != 0 || K == 0) return cudaErrorInvalidValue;
+  // The gated-residual epilogues also come in a 224-wide form; it is used
+  // when it fills the CTA pairs' waves better.
+  const bool narrow = N % 224 == 0 && wave_cost(M, N, 224) < wave_cost(M, N, 256);
   switch (epi) {
-    case EPI_STORE: return run<EPI_STORE>(M, N, K, A, Bm, e, st);
-    case EPI_QKV: return run<EPI_QKV>(M, N, K, A, Bm, e, st);
-    case EPI_RESID: return run<EPI_RESID>(M, N, K, A, Bm, e, st);
-    case EPI_SWIGLU: return run<EPI_SWIGLU>(M, N, K, A, Bm, e, st);
-    case EPI_RESID_F32: return run<EPI_RESID_F32>(M, N, K, A, Bm, e, st);
+    case EPI_STORE: return run<EPI_STORE, 256>(M, N, K, A, Bm, e, st);
+    case EPI_QKV: return run<EPI_QKV, 256>(M, N, K, A, Bm, e, st);
+    case EPI_RESID:
+      return narrow ? run<EPI_RESID, 224>(M, N, K, A, Bm, e, st)
+                    : run<EPI_RESID, 256>(M, N, K, A, Bm, e, st);
+    case EPI_SWIGLU: return run<EPI_SWIGLU, 256>(M, N, K, A, Bm, e, st);
+    case EPI_RESID_F32:
+      return narrow ? run<EPI_RESID_F32, 224>(M, N, K, A, Bm, e, st)
+                    : run<EPI_RESID_F32, 256>(M, N, K, A, Bm, e, st);
     default: return cudaErrorInvalidValue;
   }
 }
