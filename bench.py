@@ -485,6 +485,105 @@ def run_gpu(args, world, rank, local):
     return 0
 
 
+STACK_CFG = 5
+STACK_BLOCKS = 50
+STACK_WORKLOAD = ("full-width MiniMax-H3 50-block stack forward, S=16384 packed rows (15872 "
+                  "valid: text | video | audio with four 128-row padding runs), two timesteps, "
+                  "fp32 residual stream inside the stack")
+
+
+def run_stack(args):
+    """--stack: the 50-block stack forward on one GPU (layout prepared once, the
+    per-forward prologue for the two timesteps, then the stack with the valid rows
+    gathered into an fp32 stream and scattered back). Prints one JSON line with
+    the forward time, valid rows/s and TFLOP/s (algorithmic flops of 50 blocks
+    over the valid rows and the valid document)."""
+    import torch
+    from audio_generation_b200 import h3
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    dims = FULL_DIMS
+    d = h3.make_dims(dims)
+    L = config_layout(STACK_CFG)
+    S, V = L.S, L.n_valid
+
+    def to_dev_bits(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(
+            torch.bfloat16)
+
+    def to_dev_f32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+    def to_dev_i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+    keep, cws = [], []
+    for i in range(STACK_BLOCKS):
+        w = block_weights(dims, STACK_CFG, i)
+        t = {k: to_dev_bits(getattr(w, k)) for k in ("w_qkv", "q_norm", "k_norm", "w_o", "w13",
+                                                    "w2")}
+        t["ada_table"] = to_dev_f32(w.ada_table)
+        keep.append(t)
+        cws.append(h3.make_block_weights(t["w_qkv"], t["q_norm"], t["k_norm"], t["w_o"],
+                                         t["w13"], t["w2"], t["ada_table"]))
+    pw = prologue_weights(dims, STACK_CFG)
+    pos, tags, tidx = to_dev_f32(L.pos), to_dev_i32(L.tags), to_dev_i32(L.t_idx)
+    vi, ai, ti = to_dev_i32(L.video_idx), to_dev_i32(L.audio_idx), to_dev_i32(L.text_idx)
+    layout = h3.h3_layout_prepare(d, S, L.n_t, pos, tags, tidx, vi, ai, ti)
+    t_dev, w1, w2p, wp = (to_dev_f32(L.timestep), to_dev_f32(pw.w_t1), to_dev_f32(pw.w_t2),
+                          to_dev_f32(pw.w_proj))
+    tws_b = h3.h3_timestep_workspace_size(d, L.n_t)
+    tws = torch.empty(tws_b, dtype=torch.uint8, device=device)
+    tmod = torch.empty((L.n_t, 6, dims.hidden), dtype=torch.float32, device=device)
+    x_host = torch.from_numpy(activations(dims, STACK_CFG, S, 1).view(np.int16)).view(
+        torch.bfloat16)
+    x0 = x_host.to(device)
+    x = torch.empty_like(x0)
+    ws_b = h3.h3_workspace_size(d, 1, S)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def forward():
+        x.copy_(x0, non_blocking=True)
+        h3.h3_timestep_modulation(d, L.n_t, t_dev, w1, w2p, wp, tmod, tws, tws_b, stream)
+        h3.h3_stack_forward(d, cws, layout, tmod, x, 1, ws, ws_b, stream)
+
+    for _ in range(args.warmup):
+        forward()
+    torch.cuda.synchronize(device)
+    gpu_id = torch.cuda.get_device_properties(device).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        time.sleep(0.3)
+        e0.record(stream)
+        for _ in range(args.steps):
+            forward()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    if h3.h3_layout_error(layout) != h3.H3_OK:
+        raise RuntimeError("device error word set during the stack run")
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = STACK_BLOCKS * block_flops(dims, V)
+    peaks = load_peaks()
+    tflops = flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "valid packed rows/s per 50-block stack forward (bf16, 1xB200)",
+        "value": V / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights and activations)",
+        "config": {"workload": STACK_WORKLOAD, "S": S, "valid_rows": V, "blocks": STACK_BLOCKS,
+                   "n_t": int(L.n_t)},
+        "tflops": tflops, "frac_of_sustained_peak": tflops / peaks["bf16_tflops_sustained"],
+        "frac_of_burst_peak": tflops / peaks["bf16_tflops"], "clocks": clk.summary(),
+        "gpu_launches": args.steps * (4 + 2 + 7 * STACK_BLOCKS),  # prologue, gather / scatter, blocks
+    }
+    print(json.dumps(line))
+    layout.close()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -496,12 +595,16 @@ def main(argv=None):
     ap.add_argument("--ref-budget-s", type=float, default=150.0,
                     help="time box of the reference arm's timed samples")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stack", action="store_true",
+                    help="time the 50-block stack forward instead (one GPU, own JSON line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.stack:
+        return run_stack(args)
     return run_gpu(args, world, rank, local)
 
 
