@@ -314,7 +314,7 @@ h3_status h3_unpack_rows(h3_layout_t L, int B, int row_elems, const void* x_pack
 
 size_t h3_timestep_workspace_size(const h3_dims* dims, int n_t) {
   if (check_dims(dims) != H3_OK || n_t < 0) return 0;
-  return align256((size_t)n_t * (dims->freq_dim + dims->time_hidden + dims->time_embed_dim) * 4);
+  return h3::timestep_workspace_bytes(*dims, n_t, true);
 }
 
 h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const float* t, const float* w_t1,
@@ -328,8 +328,7 @@ h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const float* t, c
       !aligned16(tmod) || !aligned16(ws))
     return H3_ERR_ALIGN;
   if (ws_bytes < h3_timestep_workspace_size(dims, n_t)) return H3_ERR_WORKSPACE;
-  H3_CUDA(launch_timestep(*dims, n_t, t, w_t1, w_t2, w_proj, tmod, static_cast<float*>(ws),
-                          as_stream(stream)));
+  H3_CUDA(launch_timestep(*dims, n_t, t, w_t1, w_t2, w_proj, tmod, ws, true, as_stream(stream)));
   return H3_OK;
 }
 

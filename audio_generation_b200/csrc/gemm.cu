@@ -8,8 +8,9 @@
 // costs tens of cycles to issue whatever its size, so the pair form (twice the
 // work of a 128-row MMA per instruction) keeps the tensor core fed; it also
 // halves each SM's share of B traffic and shared-memory operand reads.
-// BN is 256, or 224 for the gated-residual GEMMs when that fills the last wave
-// of tiles better (the launcher compares waves x tile width for both).
+// BN is 256, or 224 (except for the QKV and SwiGLU epilogues) when N is not a
+// multiple of 256 or when 224 fills the last wave of tiles better (the
+// launcher compares waves x tile width for both).
 // Per CTA (6 warps):
 //   warp 0        TMA producer: 128x64 A and (BN/2)x64 B-half tiles (128-B
 //                 swizzle) into a 6-stage shared-memory ring; completion is
@@ -36,6 +37,7 @@
 //              x bf16 (EPI_RESID) or fp32 (EPI_RESID_F32, the stack's stream).
 //   EPI_SWIGLU W1 / W3 interleaved in 128-row blocks: g = SiLU(a) * b.
 //   EPI_STORE  plain bf16 store (the GEMM core on its own).
+//   EPI_F32    plain fp32 store (the prologue's split-operand GEMMs).
 #include "host_util.cuh"
 #include "internal.cuh"
 #include "sm100.cuh"
@@ -97,6 +99,19 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
       float v[32];
       ld_acc(taddr + 32 * c, v);
       if (row_ok) store_bf16x32(out + (size_t)m * N + n0 + 32 * c, v);
+    }
+  } else if constexpr (EPI == EPI_F32) {
+    float* out = reinterpret_cast<float*>(e.out);
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      float v[32];
+      ld_acc(taddr + 32 * c, v);
+      if (row_ok) {
+        float4* d = reinterpret_cast<float4*>(out + (size_t)m * N + n0 + 32 * c);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      }
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out);
@@ -412,12 +427,21 @@ long long wave_cost(int M, int N, int bn) {
 cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void* Bm,
                         const GemmEpiArgs& e, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  if (N % 256 != 0 || K % BK != 0 || K == 0) return cudaErrorInvalidValue;
-  // The gated-residual epilogues also come in a 224-wide form; it is used
-  // when it fills the CTA pairs' waves better.
-  const bool narrow = N % 224 == 0 && wave_cost(M, N, 224) < wave_cost(M, N, 256);
+  if (K % BK != 0 || K == 0) return cudaErrorInvalidValue;
+  // QKV and SwiGLU epilogues pair 128-column halves of a 256-wide tile. The
+  // others also come in a 224-wide form, used when N is not a multiple of 256
+  // or when it fills the CTA pairs' waves better.
+  const bool w256 = N % 256 == 0, w224 = N % 224 == 0;
+  if (epi == EPI_QKV || epi == EPI_SWIGLU) {
+    if (!w256) return cudaErrorInvalidValue;
+  } else if (!w256 && !w224) {
+    return cudaErrorInvalidValue;
+  }
+  const bool narrow = w224 && (!w256 || wave_cost(M, N, 224) < wave_cost(M, N, 256));
   switch (epi) {
-    case EPI_STORE: return run<EPI_STORE, 256>(M, N, K, A, Bm, e, st);
+    case EPI_STORE:
+      return narrow ? run<EPI_STORE, 224>(M, N, K, A, Bm, e, st)
+                    : run<EPI_STORE, 256>(M, N, K, A, Bm, e, st);
     case EPI_QKV: return run<EPI_QKV, 256>(M, N, K, A, Bm, e, st);
     case EPI_RESID:
       return narrow ? run<EPI_RESID, 224>(M, N, K, A, Bm, e, st)
@@ -426,6 +450,9 @@ cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void*
     case EPI_RESID_F32:
       return narrow ? run<EPI_RESID_F32, 224>(M, N, K, A, Bm, e, st)
                     : run<EPI_RESID_F32, 256>(M, N, K, A, Bm, e, st);
+    case EPI_F32:
+      return narrow ? run<EPI_F32, 224>(M, N, K, A, Bm, e, st)
+                    : run<EPI_F32, 256>(M, N, K, A, Bm, e, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -84,17 +84,29 @@ cudaError_t launch_norm_modulate(const LayoutView& L, int B, int H, int chunk_sh
                                  const float* table, const float* tmod, void* h,
                                  cudaStream_t st);
 
+// The prologue's fp32 GEMMs run either on the CUDA cores or, for many distinct
+// timesteps, as bf16 tensor-core GEMMs over three-way bf16 splits of both
+// operands (allow_split = false forces the first form). Workspace bytes for
+// either form; ws must be 256-byte aligned.
+size_t timestep_workspace_bytes(const h3_dims& d, int n_t, bool allow_split);
 cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const float* w_t1,
-                            const float* w_t2, const float* w_proj, float* tmod, float* ws,
-                            cudaStream_t st);
+                            const float* w_t2, const float* w_proj, float* tmod, void* ws,
+                            bool allow_split, cudaStream_t st);
 
 // EPI_RESID_F32: gated residual on an fp32 residual stream (inside the stack).
-enum GemmEpilogue { EPI_STORE = 0, EPI_QKV = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_RESID_F32 = 4 };
+enum GemmEpilogue {
+  EPI_STORE = 0,
+  EPI_QKV = 1,
+  EPI_RESID = 2,
+  EPI_SWIGLU = 3,
+  EPI_RESID_F32 = 4,
+  EPI_F32 = 5
+};
 
 struct GemmEpiArgs {
   LayoutView L;
   int B = 1, NH = 0;
-  // EPI_STORE: out [M, N]; EPI_SWIGLU: out [M, N/2]
+  // EPI_STORE: out [M, N] bf16; EPI_F32: out [M, N] fp32; EPI_SWIGLU: out [M, N/2]
   void* out = nullptr;
   // EPI_QKV
   void *q = nullptr, *k = nullptr, *v = nullptr;

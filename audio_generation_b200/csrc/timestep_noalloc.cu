@@ -12,9 +12,11 @@
 //
 // Limits and sharing:
 //  - The array holds kStaticScratchBytes (4 MiB); n_t is accepted only while
-//    h3_timestep_workspace_size(dims, n_t) fits in it (at the full constructor
-//    widths, n_t <= 126). Larger requests return H3_ERR_WORKSPACE before any
-//    work is queued.
+//    the scratch of the CUDA-core form of the prologue fits in it (at the full
+//    constructor widths, n_t <= 126). Larger requests return H3_ERR_WORKSPACE
+//    before any work is queued. (h3_timestep_modulation switches to
+//    tensor-core GEMMs over split operands from 256 timesteps on; this entry
+//    does not.)
 //  - Every GPU that loads the library holds its own copy of the array until the
 //    process exits.
 //  - All calls on a device share that one array, and the array keeps the last
@@ -66,9 +68,11 @@ extern "C" h3_status h3_timestep_modulation_noalloc(const h3_dims* dims, int n_t
                                                     const float* w_t1, const float* w_t2,
                                                     const float* w_proj, float* tmod,
                                                     h3_stream_t stream) {
-  const size_t need = h3_timestep_workspace_size(dims, n_t);
   if (dims == nullptr || n_t < 0) return H3_ERR_ARG;
-  if (need == 0 && n_t > 0) return H3_ERR_SHAPE;
+  if (n_t > 0 && h3_timestep_workspace_size(dims, n_t) == 0) return H3_ERR_SHAPE;
+  // This entry always runs the CUDA-core form of the prologue GEMMs (the split
+  // form's operand copies would not fit the fixed array).
+  const size_t need = h3::timestep_workspace_bytes(*dims, n_t, false);
   if (need > kStaticScratchBytes) return H3_ERR_WORKSPACE;
   if (n_t == 0) return H3_OK;
   if (!t || !w_t1 || !w_t2 || !w_proj || !tmod) return H3_ERR_ARG;
@@ -78,8 +82,7 @@ extern "C" h3_status h3_timestep_modulation_noalloc(const h3_dims* dims, int n_t
   void* scratch = nullptr;
   const h3_status s = scratch_address(&scratch);
   if (s != H3_OK) return s;
-  const cudaError_t e = h3::launch_timestep(*dims, n_t, t, w_t1, w_t2, w_proj, tmod,
-                                            static_cast<float*>(scratch),
-                                            reinterpret_cast<cudaStream_t>(stream));
+  const cudaError_t e = h3::launch_timestep(*dims, n_t, t, w_t1, w_t2, w_proj, tmod, scratch,
+                                            false, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? H3_OK : H3_ERR_CUDA;
 }

@@ -175,7 +175,11 @@ H3_API h3_status h3_unpack_rows(h3_layout_t layout, int B, int row_elems, const 
  * parameters freq_dim, time_embed_hidden_dim, time_embed_dim).
  *   t [n_t] f32, w_t1 [time_hidden, freq_dim], w_t2 [time_embed_dim, time_hidden],
  *   w_proj [6H, time_embed_dim] (all f32), tmod [n_t, 6, H] f32.
- * ws must hold h3_timestep_workspace_size(dims, n_t) bytes. */
+ * ws must hold h3_timestep_workspace_size(dims, n_t) bytes (16-byte aligned).
+ * From 256 timesteps on (when the widths allow) the three GEMMs run on the
+ * tensor cores over three-way bf16 splits of both fp32 operands, whose copies
+ * live in ws: the workspace then also holds, for the largest GEMM, n_t x 6K
+ * and N x 6K bf16 values (about 1.3 GB at n_t = 8192 and the full widths). */
 H3_API size_t h3_timestep_workspace_size(const h3_dims* dims, int n_t);
 H3_API h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const float* t, const float* w_t1,
                                  const float* w_t2, const float* w_proj, float* tmod, void* ws,
@@ -187,9 +191,9 @@ H3_API h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const floa
  * The pages have no counterpart to this entry point; it exists for those
  * callers. It allocates nothing: its scratch is a fixed 4 MiB device array
  * inside the library (one per GPU that loads the library, held until exit).
- * n_t is accepted while h3_timestep_workspace_size(dims, n_t) <= 4 MiB (n_t <= 126
- * at the full constructor widths); larger n_t returns H3_ERR_WORKSPACE before any
- * work is queued. All calls on a device share the array: calls whose work
+ * It always uses the CUDA-core form of the GEMMs; n_t is accepted while that
+ * form's scratch fits in 4 MiB (n_t <= 126 at the full constructor widths);
+ * larger n_t returns H3_ERR_WORKSPACE before any work is queued. All calls on a device share the array: calls whose work
  * overlaps on the GPU race (order them on one stream or with events). Nothing in
  * the array needs to start at zero. The first call on a device looks up the
  * array's address; make it before any stream capture. */

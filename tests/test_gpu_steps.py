@@ -171,8 +171,11 @@ def test_ffn_down_residual(case):
 TMOD_REL = 1e-4
 
 
-@pytest.mark.parametrize("dims,n_t", [(TINY_DIMS, 256), (FULL_DIMS, 3), (FULL_DIMS, 70)])
+@pytest.mark.parametrize("dims,n_t", [(TINY_DIMS, 256), (TINY_DIMS, 255), (FULL_DIMS, 3),
+                                      (FULL_DIMS, 70), (FULL_DIMS, 300)])
 def test_timestep_modulation(dims, n_t):
+    """n_t < 256: fp32 GEMMs on the CUDA cores; n_t >= 256: tensor-core GEMMs over
+    three-way bf16 splits of the fp32 operands (same fp32-level tolerance)."""
     pw = prologue_weights(dims, 1 if dims is TINY_DIMS else 2)
     g = np.random.default_rng(n_t)
     t = g.random(n_t).astype(np.float32)
@@ -187,4 +190,25 @@ def test_timestep_modulation(dims, n_t):
     torch.cuda.synchronize()
     ref = O.timestep_modulation(t, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim, dims.hidden)
     got = tmod.double().cpu().numpy()
+    assert rel_l2(got, ref) < TMOD_REL
+
+
+def test_timestep_modulation_many_timesteps_sampled_rows():
+    """2048 per-row timesteps at full width (split-operand tensor-core form):
+    rows are independent, so sampled rows are checked against the oracle run on
+    their timesteps alone."""
+    dims, n_t = FULL_DIMS, 2048
+    pw = prologue_weights(dims, 2)
+    g = np.random.default_rng(2048)
+    t = g.random(n_t).astype(np.float32)
+    d = h3.make_dims(dims)
+    ws_b = h3.h3_timestep_workspace_size(d, n_t)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+    tmod = torch.empty((n_t, 6, dims.hidden), dtype=torch.float32, device="cuda")
+    h3.h3_timestep_modulation(d, n_t, dev_f32(t), dev_f32(pw.w_t1), dev_f32(pw.w_t2),
+                              dev_f32(pw.w_proj), tmod, ws, ws_b)
+    torch.cuda.synchronize()
+    rows = np.array([0, 1, 255, 256, 1000, 2047])
+    ref = O.timestep_modulation(t[rows], pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim, dims.hidden)
+    got = tmod[torch.as_tensor(rows, device="cuda")].double().cpu().numpy()
     assert rel_l2(got, ref) < TMOD_REL
