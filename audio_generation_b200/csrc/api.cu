@@ -23,7 +23,9 @@ h3_status check_dims(const h3_dims* d) {
   if (d->heads <= 0 || d->heads % 2 != 0) return H3_ERR_SHAPE;
   if (d->ffn <= 0 || d->ffn % 128 != 0) return H3_ERR_SHAPE;
   if (d->n_modalities < 3) return H3_ERR_SHAPE;
-  if (d->freq_dim <= 0 || d->freq_dim % 2 != 0 || d->time_hidden <= 0 || d->time_embed_dim <= 0)
+  // The prologue's GEMMs read rows in 16-byte vectors.
+  if (d->freq_dim <= 0 || d->freq_dim % 4 != 0 || d->time_hidden <= 0 ||
+      d->time_hidden % 4 != 0 || d->time_embed_dim <= 0 || d->time_embed_dim % 4 != 0)
     return H3_ERR_SHAPE;
   if (!(d->norm_eps > 0.f) || !(d->qk_norm_eps > 0.f) || !(d->rope_theta > 0.f))
     return H3_ERR_ARG;

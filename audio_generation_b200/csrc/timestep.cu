@@ -13,8 +13,8 @@
 //
 // Runs once per forward for the distinct timestep values. Two forms of the
 // three fp32 GEMMs:
-//  * few timesteps: a shared-memory-tiled fp32 GEMM on the CUDA cores (the
-//    weights are read once, which dominates);
+//  * few timesteps (n_t < kSplitMinRows): a skinny fp32 kernel on the CUDA cores
+//    that streams the weights once per chunk of eight timesteps (HBM-bound);
 //  * many timesteps (n_t >= kSplitMinRows): each fp32 operand x is split into
 //    three bf16 pieces x1 = bf16(x), x2 = bf16(x - x1), x3 = bf16(x - x1 - x2)
 //    (24 significant bits, exact differences), and the six products of pieces
@@ -47,7 +47,7 @@ __global__ void k_sinusoid(int n_t, int freq_dim, const float* __restrict__ t,
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
 
-constexpr int kSplitMinRows = 256;
+constexpr int kSplitMinRows = 65;
 
 // dst[r, p K + k] = piece(p) of act(src[r, k]), p = 0..5, with pieces
 // (x1, x1, x2, x1, x2, x3) on the A side and (y1, y2, y1, y3, y2, y1) on the B
@@ -111,65 +111,79 @@ size_t stage_bytes(int n_t, int K, int N) {
   return align256((size_t)n_t * 6 * K * 2) + align256((size_t)N * 6 * K * 2);
 }
 
-// C[n, o] = sum_k act(A[n, k]) * W[o, k]; 64x64 tile, 16-wide K slices, 4x4 per thread.
-template <bool kSiluA>
-__global__ void __launch_bounds__(256) k_sgemm_nt(int N, int O, int K,
-                                                  const float* __restrict__ A,
-                                                  const float* __restrict__ W,
-                                                  float* __restrict__ C) {
-  __shared__ float As[16][64 + 4];
-  __shared__ float Ws[16][64 + 4];
-  const int tid = threadIdx.x;
-  const int n0 = blockIdx.y * 64, o0 = blockIdx.x * 64;
-  const int tr = tid / 16, tc = tid % 16;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    // 64 rows x 16 k of A and of W: 1024 values each, 4 per thread
+// C[n, o] = sum_k A[n, k] W[o, k] for few rows n: each warp streams two rows
+// of W once (16-byte loads, coalesced across the warp) against a chunk of up to
+// kSkinnyRows rows of A (small enough to stay in L1 / L2), keeps the 2 x
+// kSkinnyRows partial dot products per lane and reduces them across the warp
+// at the end. Blocks along y take successive chunks of A's rows. HBM-bound on
+// W for a handful of rows.
+constexpr int kSkinnyRows = 8;
+
+__global__ void __launch_bounds__(256) k_skinny_nt(int N, int O, int K,
+                                                   const float* __restrict__ A,
+                                                   const float* __restrict__ W,
+                                                   float* __restrict__ C) {
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.y * kSkinnyRows;
+  const int nr = min(kSkinnyRows, N - n0);
+  const int k4n = K >> 2;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long wp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       2 * wp < O; wp += warps) {
+    const int o0 = (int)(2 * wp), o1 = min(o0 + 1, O - 1);
+    const float4* w0 = reinterpret_cast<const float4*>(W + (size_t)o0 * K);
+    const float4* w1 = reinterpret_cast<const float4*>(W + (size_t)o1 * K);
+    float acc0[kSkinnyRows] = {}, acc1[kSkinnyRows] = {};
+    for (int k4 = lane; k4 < k4n; k4 += 32) {
+      const float4 a0 = __ldg(w0 + k4), a1 = __ldg(w1 + k4);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int e = tid + 256 * q;
-      const int r = e / 16, kk = e % 16;
-      float a = 0.f, w = 0.f;
-      if (n0 + r < N && k0 + kk < K) {
-        a = A[(size_t)(n0 + r) * K + k0 + kk];
-        if (kSiluA) a = silu_f(a);
+      for (int r = 0; r < kSkinnyRows; ++r) {
+        if (r < nr) {
+          const float4 x = __ldg(reinterpret_cast<const float4*>(A + (size_t)(n0 + r) * K) + k4);
+          acc0[r] = fmaf(a0.x, x.x, fmaf(a0.y, x.y, fmaf(a0.z, x.z, fmaf(a0.w, x.w, acc0[r]))));
+          acc1[r] = fmaf(a1.x, x.x, fmaf(a1.y, x.y, fmaf(a1.z, x.z, fmaf(a1.w, x.w, acc1[r]))));
+        }
       }
-      if (o0 + r < O && k0 + kk < K) w = W[(size_t)(o0 + r) * K + k0 + kk];
-      As[kk][r] = a;
-      Ws[kk][r] = w;
     }
-    __syncthreads();
 #pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], w[4];
+    for (int r = 0; r < kSkinnyRows; ++r) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][tr * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) w[j] = Ws[kk][tc * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+      for (int off = 16; off; off >>= 1) {
+        acc0[r] += __shfl_xor_sync(0xffffffffu, acc0[r], off);
+        acc1[r] += __shfl_xor_sync(0xffffffffu, acc1[r], off);
+      }
     }
-    __syncthreads();
-  }
+    if (lane == 0) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int n = n0 + tr * 4 + i;
-    if (n >= N) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int o = o0 + tc * 4 + j;
-      if (o < O) C[(size_t)n * O + o] = acc[i][j];
+      for (int r = 0; r < kSkinnyRows; ++r) {
+        if (r < nr) {
+          C[(size_t)(n0 + r) * O + o0] = acc0[r];
+          if (o1 != o0) C[(size_t)(n0 + r) * O + o1] = acc1[r];
+        }
+      }
     }
   }
 }
 
-template <bool kSilu>
-cudaError_t sgemm(int N, int O, int K, const float* A, const float* W, float* C,
-                  cudaStream_t st) {
-  dim3 grid((O + 63) / 64, (N + 63) / 64);
-  k_sgemm_nt<kSilu><<<grid, 256, 0, st>>>(N, O, K, A, W, C);
+__global__ void k_silu_inplace(size_t n, float* __restrict__ x) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    x[i] = silu_f(x[i]);
+}
+
+cudaError_t skinny(int N, int O, int K, const float* A, const float* W, float* C,
+                   cudaStream_t st) {
+  const int chunks = (N + kSkinnyRows - 1) / kSkinnyRows;
+  int gx = (O / 2 + 7) / 8;  // eight warps (two rows of W each) per block
+  if (gx > 4 * 148 * 8) gx = 4 * 148 * 8;
+  k_skinny_nt<<<dim3(gx, chunks), 256, 0, st>>>(N, O, K, A, W, C);
+  return cudaGetLastError();
+}
+
+cudaError_t silu_inplace(size_t n, float* x, cudaStream_t st) {
+  size_t grid = (n + 255) / 256;
+  if (grid > 16384) grid = 16384;
+  k_silu_inplace<<<(unsigned)grid, 256, 0, st>>>(n, x);
   return cudaGetLastError();
 }
 
@@ -200,12 +214,13 @@ cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const flo
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   if (!use_split(d, n_t, allow_split)) {
-    if ((err = sgemm<false>(n_t, d.time_hidden, d.freq_dim, e, w_t1, h1, st)) != cudaSuccess)
+    // SiLU is applied once, in place, to each GEMM's input activations.
+    if ((err = skinny(n_t, d.time_hidden, d.freq_dim, e, w_t1, h1, st)) != cudaSuccess) return err;
+    if ((err = silu_inplace((size_t)n_t * d.time_hidden, h1, st)) != cudaSuccess) return err;
+    if ((err = skinny(n_t, d.time_embed_dim, d.time_hidden, h1, w_t2, temb, st)) != cudaSuccess)
       return err;
-    if ((err = sgemm<true>(n_t, d.time_embed_dim, d.time_hidden, h1, w_t2, temb, st)) !=
-        cudaSuccess)
-      return err;
-    return sgemm<true>(n_t, 6 * d.hidden, d.time_embed_dim, temb, w_proj, tmod, st);
+    if ((err = silu_inplace((size_t)n_t * d.time_embed_dim, temb, st)) != cudaSuccess) return err;
+    return skinny(n_t, 6 * d.hidden, d.time_embed_dim, temb, w_proj, tmod, st);
   }
   // Split operands of one stage at a time, after the fp32 activations.
   uint8_t* stage = static_cast<uint8_t*>(ws) +

@@ -15,7 +15,7 @@
 //    the scratch of the CUDA-core form of the prologue fits in it (at the full
 //    constructor widths, n_t <= 126). Larger requests return H3_ERR_WORKSPACE
 //    before any work is queued. (h3_timestep_modulation switches to
-//    tensor-core GEMMs over split operands from 256 timesteps on; this entry
+//    tensor-core GEMMs over split operands from 65 timesteps on; this entry
 //    does not.)
 //  - Every GPU that loads the library holds its own copy of the array until the
 //    process exits.

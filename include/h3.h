@@ -176,7 +176,7 @@ H3_API h3_status h3_unpack_rows(h3_layout_t layout, int B, int row_elems, const 
  *   t [n_t] f32, w_t1 [time_hidden, freq_dim], w_t2 [time_embed_dim, time_hidden],
  *   w_proj [6H, time_embed_dim] (all f32), tmod [n_t, 6, H] f32.
  * ws must hold h3_timestep_workspace_size(dims, n_t) bytes (16-byte aligned).
- * From 256 timesteps on (when the widths allow) the three GEMMs run on the
+ * From 65 timesteps on (when the widths allow) the three GEMMs run on the
  * tensor cores over three-way bf16 splits of both fp32 operands, whose copies
  * live in ws: the workspace then also holds, for the largest GEMM, n_t x 6K
  * and N x 6K bf16 values (about 1.3 GB at n_t = 8192 and the full widths). */

@@ -71,7 +71,7 @@ def _a256(n):
 
 def _tmod_ws_expected(dims, n_t):
     base = _a256(n_t * (dims.freq_dim + dims.time_hidden + dims.time_embed_dim) * 4)
-    if n_t < 256:
+    if n_t < 65:
         return base
     stages = [(dims.freq_dim, dims.time_hidden), (dims.time_hidden, dims.time_embed_dim),
               (dims.time_embed_dim, 6 * dims.hidden)]
@@ -79,15 +79,17 @@ def _tmod_ws_expected(dims, n_t):
 
 
 @pytest.mark.parametrize("dims", [TINY_DIMS, FULL_DIMS])
-@pytest.mark.parametrize("n_t", [0, 1, 3, 126, 255, 256, 8192])
+@pytest.mark.parametrize("n_t", [0, 1, 3, 64, 65, 126, 256, 8192])
 def test_timestep_workspace_size(dims, n_t):
-    """CUDA-core form below 256 timesteps (three fp32 activations); from 256 on
+    """CUDA-core form below 65 timesteps (three fp32 activations); from 65 on
     also the bf16 split copies of the largest GEMM's two operands."""
     assert h3.h3_timestep_workspace_size(h3.make_dims(dims), n_t) == _tmod_ws_expected(dims, n_t)
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 64), ("hidden", 500), ("heads", 5),
-                                         ("ffn", 1000), ("rope_freq_dim", 8)])
+                                         ("ffn", 1000), ("rope_freq_dim", 8),
+                                         ("freq_dim", 258), ("time_hidden", 5378),
+                                         ("time_embed_dim", 2690)])
 def test_unsupported_dims_are_rejected_on_the_host(field, value):
     kw = dict(FULL_DIMS.__dict__)
     kw[field] = value

@@ -171,11 +171,13 @@ def test_ffn_down_residual(case):
 TMOD_REL = 1e-4
 
 
-@pytest.mark.parametrize("dims,n_t", [(TINY_DIMS, 256), (TINY_DIMS, 255), (FULL_DIMS, 3),
-                                      (FULL_DIMS, 70), (FULL_DIMS, 300)])
+@pytest.mark.parametrize("dims,n_t", [(TINY_DIMS, 256), (TINY_DIMS, 64), (TINY_DIMS, 65),
+                                      (FULL_DIMS, 2), (FULL_DIMS, 3), (FULL_DIMS, 17),
+                                      (FULL_DIMS, 64), (FULL_DIMS, 70), (FULL_DIMS, 300)])
 def test_timestep_modulation(dims, n_t):
-    """n_t < 256: fp32 GEMMs on the CUDA cores; n_t >= 256: tensor-core GEMMs over
-    three-way bf16 splits of the fp32 operands (same fp32-level tolerance)."""
+    """n_t < 65: skinny fp32 GEMMs on the CUDA cores (chunks of eight timesteps,
+    ragged last chunk at 17); n_t >= 65: tensor-core GEMMs over three-way bf16
+    splits of the fp32 operands (same fp32-level tolerance)."""
     pw = prologue_weights(dims, 1 if dims is TINY_DIMS else 2)
     g = np.random.default_rng(n_t)
     t = g.random(n_t).astype(np.float32)
