@@ -59,3 +59,31 @@ def test_work_counts_match_the_stated_flops():
     assert abs(f - (2 * 8192 * (5376 * 21504 + 7168 * 5376 + 5376 * 28672 + 14336 * 5376)
                     + 4 * 56 * 128 * 8192 ** 2)) < 1
     assert abs(f / 1e12 - 8.238) < 0.01
+
+
+def test_recorded_traffic_is_used_only_for_the_recorded_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu summary only while the
+    kernel's source file still hashes to the recorded SHA-256."""
+    import hashlib
+    src = tmp_path / "k.cu"
+    src.write_text("// a kernel\n")
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()
+    rec = tmp_path / "traffic.txt"
+    rec.write_text(f"# comment line\nattention {digest} 123456\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setitem(bench.KERNEL_SOURCES, "attention", "k.cu")
+    (tmp_path / "audio_generation_b200" / "csrc").mkdir(parents=True)
+    (tmp_path / "audio_generation_b200" / "csrc" / "k.cu").write_bytes(src.read_bytes())
+    assert bench.measured_traffic("attention") == 123456.0
+    (tmp_path / "audio_generation_b200" / "csrc" / "k.cu").write_text("// changed\n")
+    assert bench.measured_traffic("attention") is None
+
+
+def test_algorithmic_bytes_per_kernel():
+    from workloads import FULL_DIMS
+    b = bench.kernel_bytes(FULL_DIMS, 8192)
+    H, A, F, V = 5376, 7168, 14336, 8192
+    assert b["attention"] == 4 * V * A * 2
+    assert b["ffn_up"] == V * H * 2 + 2 * F * H * 2 + V * F * 2
+    assert b["norm_modulate_1"] == V * 12 * H
