@@ -25,6 +25,14 @@ CASES = {
     "full_rand300": (FULL_DIMS, lambda: random_layout(300, 6, pad_runs=2, max_run=50), 1),
     "tiny_rand1500": (TINY_DIMS, lambda: random_layout(1500, 7, pad_runs=4, max_run=300), 1),
 }
+# Attention-only cases at full width with more work items (pairs of query tiles
+# x 56 heads) than one wave of the GPU; "full_sparse1500" keeps only two key
+# tiles and has all-padding pairs of query tiles.
+ATTN_CASES = {
+    "full_rand1500": (FULL_DIMS, lambda: random_layout(1500, 8, pad_runs=3, max_run=200), 1),
+    "full_sparse1500": (FULL_DIMS, lambda: make_layout([("text", 0, 100), ("pad", 1372),
+                                                        ("audio", 0, 28)]), 1),
+}
 
 
 def _tmod(n_t, H, seed, std=0.5):
@@ -87,9 +95,16 @@ def _attention_inputs(dims, L, B, seed, q_scale=1.0):
 
 @pytest.mark.parametrize("case,q_scale", [("tiny_cfg1_B2", 1.0), ("tiny_rand333", 1.0),
                                           ("tiny_rand333", 6.0), ("full_rand300", 1.0),
-                                          ("tiny_rand1500", 1.0), ("tiny_rand1500", 6.0)])
+                                          ("tiny_rand1500", 1.0), ("tiny_rand1500", 6.0),
+                                          ("full_rand1500", 1.0), ("full_sparse1500", 1.0),
+                                          ("full_sparse1500", 6.0)])
 def test_attention(case, q_scale):
-    dims, L, dl, w, B = _setup(case)
+    if case in ATTN_CASES:
+        dims, mk, B = ATTN_CASES[case]
+        L = mk()
+        dl = DevLayout(dims, L)
+    else:
+        dims, L, dl, w, B = _setup(case)
     NH, D = dims.heads, dims.head_dim
     qb, kb, vb = _attention_inputs(dims, L, B, 11, q_scale)
     o = torch.full((B, L.S, NH * D), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -104,6 +119,7 @@ def test_attention(case, q_scale):
         ref = O.attention(t(qb), pad, t(kb), t(vb), pad)
         assert_close(got[b, ~pad], ref[~pad], what=f"attention b={b}", storage_rounding=True)
         assert np.all(got[b, allpad_rows] == 0.0)
+    assert np.all(np.isfinite(got))
 
 
 @pytest.mark.parametrize("case", list(CASES))
