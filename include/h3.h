@@ -29,8 +29,9 @@
  *    h3_layout_export only enqueues work and returns; argument, shape and
  *    alignment errors are returned synchronously before anything is launched.
  *  - Alignment: every device pointer must be 16-byte aligned.
- *  - Shapes: head_dim == 128; hidden % 256 == 0; heads even; ffn % 128 == 0;
- *    rope_freq_dim == 16; time dims % 4 == 0. S (rows) is arbitrary >= 0.
+ *  - Shapes: head_dim == 128; hidden % 256 == 0 and <= 6144; heads even;
+ *    ffn % 128 == 0; rope_freq_dim == 16; freq_dim, time_hidden and
+ *    time_embed_dim % 4 == 0. S (rows) is arbitrary >= 0.
  *  - Batch: B >= 1 elements share one layout; each element is its own attention
  *    document set (the page's "pure replication axis").
  *  - Asynchronous failures: every wait inside a kernel is bounded (about 2 s).
@@ -256,9 +257,11 @@ H3_API h3_status h3_block_forward(const h3_dims* dims, const h3_block_weights* w
 
 /* n_blocks blocks (weights: HOST array of n_blocks structs holding device
  * pointers) sharing one tmod, in place on x [B, S, H] bf16. Valid rows are
- * gathered once into a compact [B, V, H] stream (padding rows never reach a
- * valid row's result, so the blocks then run with no mask), and scattered back
- * at the end; padding rows of x are untouched. */
+ * gathered once into a compact [B, V, H] f32 stream (padding rows never reach a
+ * valid row's result, so the blocks then run with no mask); the residual stream
+ * stays f32 across the blocks and is rounded to bf16 once when scattered back
+ * at the end; padding rows of x are untouched. ws: h3_workspace_size(dims, B, S)
+ * bytes. */
 H3_API h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* weights, int n_blocks,
                            h3_layout_t layout, const float* tmod, void* x, int B, void* ws,
                            size_t ws_bytes, h3_stream_t stream);
