@@ -8,13 +8,7 @@
 
 using namespace h3;
 
-namespace {
-
-inline cudaStream_t as_stream(h3_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
-
-inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-inline size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+namespace h3 {
 
 h3_status check_dims(const h3_dims* d) {
   if (!d) return H3_ERR_ARG;
@@ -29,6 +23,24 @@ h3_status check_dims(const h3_dims* d) {
     return H3_ERR_SHAPE;
   if (!(d->norm_eps > 0.f) || !(d->qk_norm_eps > 0.f) || !(d->rope_theta > 0.f))
     return H3_ERR_ARG;
+  return H3_OK;
+}
+
+}  // namespace h3
+
+namespace {
+
+inline cudaStream_t as_stream(h3_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+// B batch elements of the layout's S rows: B * S rows must fit an int and B the
+// attention grid.
+h3_status check_batch(const h3_layout* L, int B) {
+  if (!L || B < 0) return H3_ERR_ARG;
+  if (B > kMaxBatch || (long long)B * L->S > 0x7fffffffLL) return H3_ERR_SHAPE;
   return H3_OK;
 }
 
@@ -154,6 +166,7 @@ h3_status h3_layout_prepare(const h3_dims* dims, const h3_layout_desc* desc, h3_
   const int S = desc->S;
   if (S < 0 || desc->n_t < 0 || desc->n_video < 0 || desc->n_audio < 0 || desc->n_text < 0)
     return H3_ERR_ARG;
+  if (S > kMaxRows) return H3_ERR_SHAPE;
   if (S > 0 && (!desc->pos || !desc->tags || !desc->t_idx)) return H3_ERR_ARG;
   if ((desc->n_video && !desc->video_idx) || (desc->n_audio && !desc->audio_idx) ||
       (desc->n_text && !desc->text_idx))
@@ -296,6 +309,7 @@ size_t h3_workspace_size(const h3_dims* dims, int B, int S) {
 h3_status h3_pack_rows(h3_layout_t L, int B, int row_elems, const void* video, const void* audio,
                        const void* text, void* x_packed, h3_stream_t stream) {
   if (!L || B < 0 || row_elems <= 0 || !x_packed) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   if (row_elems % 8 != 0) return H3_ERR_SHAPE;
   if ((L->n_video && !video) || (L->n_audio && !audio) || (L->n_text && !text)) return H3_ERR_ARG;
   if (!aligned16(video) || !aligned16(audio) || !aligned16(text) || !aligned16(x_packed))
@@ -307,6 +321,7 @@ h3_status h3_pack_rows(h3_layout_t L, int B, int row_elems, const void* video, c
 h3_status h3_unpack_rows(h3_layout_t L, int B, int row_elems, const void* x_packed, void* video,
                          void* audio, void* text, h3_stream_t stream) {
   if (!L || B < 0 || row_elems <= 0 || !x_packed) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   if (row_elems % 8 != 0) return H3_ERR_SHAPE;
   if (!aligned16(video) || !aligned16(audio) || !aligned16(text) || !aligned16(x_packed))
     return H3_ERR_ALIGN;
@@ -340,6 +355,7 @@ h3_status h3_norm_modulate(const h3_dims* dims, h3_layout_t L, int B, int which,
   H3_TRY(check_dims(dims));
   if (!L || B < 0 || (which != 0 && which != 1) || !x || !ada_table || !tmod || !h)
     return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   if (!aligned16(x) || !aligned16(ada_table) || !aligned16(tmod) || !aligned16(h))
     return H3_ERR_ALIGN;
   const int c0 = which == 0 ? 0 : 3;
@@ -353,6 +369,7 @@ h3_status h3_qkv_rope(const h3_dims* dims, h3_layout_t L, int B, const void* h, 
                       h3_stream_t stream) {
   H3_TRY(check_dims(dims));
   if (!L || B < 0 || !h || !w_qkv || !q_norm || !k_norm || !q || !k || !v) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   if (!aligned16(h) || !aligned16(w_qkv) || !aligned16(q_norm) || !aligned16(k_norm) ||
       !aligned16(q) || !aligned16(k) || !aligned16(v))
     return H3_ERR_ALIGN;
@@ -375,6 +392,7 @@ h3_status h3_attention(const h3_dims* dims, h3_layout_t L, int B, const void* q,
                        const void* v, void* o, h3_stream_t stream) {
   H3_TRY(check_dims(dims));
   if (!L || B < 0 || !q || !k || !v || !o) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return H3_ERR_ALIGN;
   H3_CUDA(launch_attention(L->view(), B, dims->heads, q, k, v, o, as_stream(stream)));
   return H3_OK;
@@ -385,6 +403,7 @@ h3_status h3_out_residual(const h3_dims* dims, h3_layout_t L, int B, const void*
                           h3_stream_t stream) {
   H3_TRY(check_dims(dims));
   if (!L || B < 0 || !o || !w_o || !ada_table || !tmod || !x) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   if (!aligned16(o) || !aligned16(w_o) || !aligned16(ada_table) || !aligned16(tmod) ||
       !aligned16(x))
     return H3_ERR_ALIGN;
@@ -404,6 +423,7 @@ h3_status h3_ffn_up(const h3_dims* dims, h3_layout_t L, int B, const void* h2, c
                     void* g, h3_stream_t stream) {
   H3_TRY(check_dims(dims));
   if (!L || B < 0 || !h2 || !w13 || !g) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   if (!aligned16(h2) || !aligned16(w13) || !aligned16(g)) return H3_ERR_ALIGN;
   GemmEpiArgs sg;
   sg.L = L->view();
@@ -418,6 +438,7 @@ h3_status h3_ffn_down_residual(const h3_dims* dims, h3_layout_t L, int B, const 
                                void* x, h3_stream_t stream) {
   H3_TRY(check_dims(dims));
   if (!L || B < 0 || !g || !w2 || !ada_table || !tmod || !x) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   if (!aligned16(g) || !aligned16(w2) || !aligned16(ada_table) || !aligned16(tmod) ||
       !aligned16(x))
     return H3_ERR_ALIGN;
@@ -437,6 +458,7 @@ h3_status h3_block_forward(const h3_dims* dims, const h3_block_weights* weights,
                            h3_stream_t stream) {
   H3_TRY(check_dims(dims));
   if (!L || B < 0 || !tmod || !x || !ws) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   H3_TRY(check_weights(weights));
   if (!aligned16(tmod) || !aligned16(x) || !aligned16(ws)) return H3_ERR_ALIGN;
   if (ws_bytes < h3_workspace_size(dims, B, L->S)) return H3_ERR_WORKSPACE;
@@ -451,6 +473,7 @@ h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* weights,
   H3_TRY(check_dims(dims));
   if (!L || B < 0 || n_blocks < 0 || !tmod || !x || !ws || (n_blocks > 0 && !weights))
     return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
   for (int i = 0; i < n_blocks; ++i) H3_TRY(check_weights(&weights[i]));
   if (!aligned16(tmod) || !aligned16(x) || !aligned16(ws)) return H3_ERR_ALIGN;
   if (ws_bytes < h3_workspace_size(dims, B, L->S)) return H3_ERR_WORKSPACE;

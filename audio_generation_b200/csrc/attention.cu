@@ -52,7 +52,7 @@ constexpr float kLazyRescale = 8.0f;  // log2 units
 constexpr int OFF_Q = 0, OFF_K = 2 * TILE_BYTES, OFF_V = 4 * TILE_BYTES;
 constexpr int OFF_BAR = 6 * TILE_BYTES;
 constexpr int OFF_LIST = OFF_BAR + 256;
-constexpr int kMaxKeyTiles = 4096;  // S <= 524288 rows
+constexpr int kMaxKeyTiles = kMaxRows / 128;  // the key-tile list below (S <= kMaxRows)
 constexpr int SMEM_BYTES = OFF_LIST + 2 * kMaxKeyTiles + 1024;
 
 struct Bars {
@@ -70,9 +70,10 @@ __device__ __forceinline__ float exp2_mufu(float x) {
 // 2^x on the FMA pipe: split x = j + f with j = round(x) (adding 1.5 * 2^23
 // leaves the rounded integer in the low mantissa bits) and f in [-1/2, 1/2];
 // 2^f by a cubic fitted by least squares (relative error weighted) at 256
-// Chebyshev nodes of [-1/2, 1/2], max relative error 7.7e-5 (bf16 keeps 3.9e-3);
-// j is added to the exponent field. Inputs below -126 are clamped (the result
-// is then < 2^-125, negligible next to the row sum, which is >= 1).
+// Chebyshev nodes of [-1/2, 1/2], max relative error 7.7e-5 wherever 2^x is a
+// normal float (x >= -125; bf16 keeps 3.9e-3); j is added to the exponent
+// field. Inputs below -126 are clamped; below -125 the result is off by less
+// than 2^-135 in absolute terms, negligible next to the row sum, which is >= 1.
 __device__ __forceinline__ float exp2_poly(float x) {
   x = fmaxf(x, -126.f);
   const float t = x + 12582912.f;
@@ -431,6 +432,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, const void* k,
                              const void* v, void* o, cudaStream_t st) {
   if (L.S == 0 || B == 0) return cudaSuccess;
+  if (L.n_tiles > kMaxKeyTiles || B > kMaxBatch) return cudaErrorInvalidValue;
   cudaError_t err =
       cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (err != cudaSuccess) return err;

@@ -36,6 +36,50 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Unique id of the current context (cuCtxGetId), 0 if it cannot be read.
+static unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+h3_status symbol_address(SymbolAddressCache& cache, cudaError_t (*lookup)(void**), void** out) {
+  static std::mutex m;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return H3_ERR_CUDA;
+  if (dev < 0 || dev >= SymbolAddressCache::kMaxDevices) return H3_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(m);
+  // Before the device's first runtime call there is no current context (id 0);
+  // the lookup itself makes the primary context current, so the id is read again.
+  unsigned long long ctx = current_context_id();
+  if (cache.address[dev] == nullptr || ctx == 0 || cache.context_id[dev] != ctx) {
+    void* p = nullptr;
+    if (lookup(&p) != cudaSuccess || p == nullptr) return H3_ERR_CUDA;
+    cache.address[dev] = p;
+    cache.context_id[dev] = current_context_id();
+  }
+  *out = cache.address[dev];
+  return H3_OK;
+}
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();

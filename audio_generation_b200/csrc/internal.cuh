@@ -12,6 +12,13 @@
 namespace h3 {
 
 constexpr int kTile = 128;        // row tile (attention q/kv tiles, GEMM M tile)
+// Rows of one packed sequence: the attention kernel keeps the list of key tiles
+// it visits in shared memory (kMaxRows / 128 entries), and the layout step
+// packs a row index into 28 bits.
+constexpr int kMaxRows = 524288;
+static_assert(kMaxRows < (1 << 28), "row index must fit the layout step's 28-bit field");
+// Batch elements: the attention grid's z extent, and B * S must fit an int.
+constexpr int kMaxBatch = 65535;
 constexpr int kRopeFreqs = 16;    // rope_freq_dim supported by the kernels
 constexpr int kRopePairs = 3 * kRopeFreqs;  // (cos, sin) entries per row
 
@@ -127,5 +134,20 @@ cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, 
                              const void* v, void* o, cudaStream_t st);
 
 int num_sms();
+
+// Shape checks shared by the entry points (H3_OK or the status to return).
+h3_status check_dims(const h3_dims* d);
+
+// Device address of a file-scope __device__ symbol on the current device, looked
+// up once per device and again whenever the device's context changes (after a
+// cudaDeviceReset the module is loaded anew, possibly at another address).
+// `lookup` calls cudaGetSymbolAddress in the translation unit that defines the
+// symbol.
+struct SymbolAddressCache {
+  static constexpr int kMaxDevices = 64;
+  unsigned long long context_id[kMaxDevices] = {};
+  void* address[kMaxDevices] = {};
+};
+h3_status symbol_address(SymbolAddressCache& cache, cudaError_t (*lookup)(void**), void** out);
 
 }  // namespace h3

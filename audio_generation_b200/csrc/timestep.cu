@@ -30,6 +30,15 @@
 namespace h3 {
 namespace {
 
+// Error word of the split form's GEMMs (which have no layout object): a wait
+// that runs out records H3_DEVERR_TIMEOUT here; h3_timestep_error reads and
+// clears it. One int per GPU that loads the library.
+static __device__ int g_prologue_err;
+
+SymbolAddressCache g_err_cache;
+
+cudaError_t lookup_err(void** p) { return cudaGetSymbolAddress(p, g_prologue_err); }
+
 __global__ void k_sinusoid(int n_t, int freq_dim, const float* __restrict__ t,
                            float* __restrict__ e) {
   const int half = freq_dim / 2;
@@ -223,6 +232,8 @@ cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const flo
     return skinny(n_t, 6 * d.hidden, d.time_embed_dim, temb, w_proj, tmod, st);
   }
   // Split operands of one stage at a time, after the fp32 activations.
+  void* err_word = nullptr;
+  if (symbol_address(g_err_cache, lookup_err, &err_word) != H3_OK) return cudaErrorUnknown;
   uint8_t* stage = static_cast<uint8_t*>(ws) +
                    align256((size_t)n_t * (d.freq_dim + d.time_hidden + d.time_embed_dim) * 4);
   auto gemm_stage = [&](int K, int N, const float* a, bool silu_a, const float* w,
@@ -234,7 +245,7 @@ cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const flo
     if (e2 != cudaSuccess) return e2;
     if ((e2 = split3<false, true>(N, K, w, bs, st)) != cudaSuccess) return e2;
     GemmEpiArgs ea{};
-    ea.L.err = nullptr;
+    ea.L.err = static_cast<int*>(err_word);
     ea.out = out;
     return launch_gemm(EPI_F32, n_t, N, 6 * K, as, bs, ea, st);
   };
@@ -245,3 +256,13 @@ cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const flo
 }
 
 }  // namespace h3
+
+extern "C" h3_status h3_timestep_error(void) {
+  void* p = nullptr;
+  if (h3::symbol_address(h3::g_err_cache, h3::lookup_err, &p) != H3_OK) return H3_ERR_CUDA;
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return H3_ERR_CUDA;
+  if (cudaMemcpy(&v, p, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return H3_ERR_CUDA;
+  if (v != 0 && cudaMemset(p, 0, 4) != cudaSuccess) return H3_ERR_CUDA;
+  return v == 0 ? H3_OK : H3_ERR_TIMEOUT;
+}

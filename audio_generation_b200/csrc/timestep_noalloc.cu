@@ -26,39 +26,25 @@
 //    on one stream or with events.
 //  - The first call on a device looks up the array's device address
 //    (cudaGetSymbolAddress, with that device current); make that first call
-//    before any stream capture.
-#include <mutex>
-
+//    before any stream capture. The address is looked up again when the
+//    device's context has changed since (after a cudaDeviceReset).
 #include "internal.cuh"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = 4u << 20;
-constexpr int kMaxDevices = 64;
 
 // File-scope device scratch. In host code this name is only a stand-in for the
 // symbol, never a usable address: kernels receive the device address obtained
 // from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_timestep_scratch[kStaticScratchBytes];
 
-std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+// The array's device address, looked up with the device current on the first
+// call on that device, and again if the device's context has been replaced
+// since (cudaDeviceReset loads the module anew, possibly at another address).
+h3::SymbolAddressCache g_scratch_cache;
 
-// Device address of the scratch array on the current device (set up once per device).
-h3_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return H3_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return H3_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_timestep_scratch);
-    if (e != cudaSuccess || p == nullptr) return H3_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
-  return H3_OK;
-}
+cudaError_t lookup_scratch(void** p) { return cudaGetSymbolAddress(p, g_timestep_scratch); }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -68,8 +54,10 @@ extern "C" h3_status h3_timestep_modulation_noalloc(const h3_dims* dims, int n_t
                                                     const float* w_t1, const float* w_t2,
                                                     const float* w_proj, float* tmod,
                                                     h3_stream_t stream) {
-  if (dims == nullptr || n_t < 0) return H3_ERR_ARG;
-  if (n_t > 0 && h3_timestep_workspace_size(dims, n_t) == 0) return H3_ERR_SHAPE;
+  // Same checks, in the same order, as h3_timestep_modulation.
+  const h3_status dims_ok = h3::check_dims(dims);
+  if (dims_ok != H3_OK) return dims_ok;
+  if (n_t < 0) return H3_ERR_ARG;
   // This entry always runs the CUDA-core form of the prologue GEMMs (the split
   // form's operand copies would not fit the fixed array).
   const size_t need = h3::timestep_workspace_bytes(*dims, n_t, false);
@@ -80,7 +68,7 @@ extern "C" h3_status h3_timestep_modulation_noalloc(const h3_dims* dims, int n_t
       !aligned16(tmod))
     return H3_ERR_ALIGN;
   void* scratch = nullptr;
-  const h3_status s = scratch_address(&scratch);
+  const h3_status s = h3::symbol_address(g_scratch_cache, lookup_scratch, &scratch);
   if (s != H3_OK) return s;
   const cudaError_t e = h3::launch_timestep(*dims, n_t, t, w_t1, w_t2, w_proj, tmod, scratch,
                                             false, reinterpret_cast<cudaStream_t>(stream));

@@ -72,6 +72,7 @@ _SIGNATURES = {
     "h3_timestep_workspace_size": (_sz, [ctypes.POINTER(h3_dims), _i]),
     "h3_timestep_modulation": (_i, [ctypes.POINTER(h3_dims), _i, _vp, _vp, _vp, _vp, _vp, _vp,
                                     _sz, _vp]),
+    "h3_timestep_error": (_i, []),
     "h3_timestep_modulation_noalloc": (_i, [ctypes.POINTER(h3_dims), _i, _vp, _vp, _vp, _vp,
                                             _vp, _vp]),
     "h3_norm_modulate": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _i, _vp, _vp, _vp, _vp, _vp]),
@@ -235,6 +236,10 @@ def h3_timestep_modulation(dims: h3_dims, n_t: int, t, w_t1, w_t2, w_proj, tmod,
     _check(lib().h3_timestep_modulation(ctypes.byref(dims), n_t, _ptr(t), _ptr(w_t1),
                                         _ptr(w_t2), _ptr(w_proj), _ptr(tmod), _ptr(ws),
                                         ws_bytes, _stream(stream)), "h3_timestep_modulation")
+
+
+def h3_timestep_error() -> int:
+    return lib().h3_timestep_error()
 
 
 def h3_timestep_modulation_noalloc(dims: h3_dims, n_t: int, t, w_t1, w_t2, w_proj, tmod,

@@ -1,23 +1,30 @@
 #!/usr/bin/env python
 """Benchmark: packed rows/s of one MiniMax-H3 transformer-block forward on B200.
 
-Workload: the full-width single block over the 8192-row packed sequence
-(512 text | 6144 video rows of a (6, 32, 32) grid | 1536 audio rows, no
-padding), hidden 5376, 56 heads x 128, ffn 14336, one timestep per row,
-random-init bf16 weights ~N(0, 0.02) (synthetic data; no checkpoint).
+Default workload: the full-width single block over the 32768-row packed
+sequence (512 text | 30720 video rows of a (30, 32, 32) grid | 1536 audio
+rows, no padding), hidden 5376, 56 heads x 128, ffn 14336, one timestep per
+row, random-init bf16 weights ~N(0, 0.02) (synthetic data; no checkpoint): the
+largest single-block workload, where attention is 55% of the block's flops.
+``--workload 2`` / ``--workload 3`` select the 8192-row and the padded
+16384-row blocks instead.
 
 A step is one block forward (norm+modulate, QKV + QK-norm + RoPE, attention,
 O-projection + gated residual, norm+modulate, W1/W3 + SiLU gate, W2 + gated
 residual), in place on the packed hidden stream. The per-forward prologue
 (timestep MLP + AdaLN projection) and the layout step run once, before timing.
+The line also carries the attention kernel timed alone on the padded
+16384-row layout (masked attention: padding rows form their own document),
+with its fraction of peak over the valid work.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--impl reference]
 
 N > 1 runs under torch.distributed.run, one process per GPU; every rank runs
 its own replica of the workload (the batch axis is a pure replication axis,
 so there is no data-path collective) and the reported time is the maximum
-over ranks. ``--impl reference`` times the CPU oracle on a bounded sample of
-the same workload instead.
+over ranks. ``--impl reference`` times the CPU oracle on bounded samples of
+the same workload instead: each step is a sample of query rows run through the
+float64 block, with the keys and values of every row formed once beforehand.
 """
 
 from __future__ import annotations
@@ -38,14 +45,21 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from workloads import (FULL_DIMS, activations, block_weights, config_layout,  # noqa: E402
-                       prologue_weights, make_layout)
+                       prologue_weights)
 
 METRIC = "packed rows/s per DiT block fwd (bf16, 1xB200); % of dense bf16 TC peak"
 UNIT = "rows/s"
-CFG = 2
-WORKLOAD = ("full-width MiniMax-H3 block, S=8192 packed rows (512 text | 6144 video "
-            "(6,32,32) | 1536 audio), no padding, hidden 5376, 56x128 heads, ffn 14336, "
-            "per-row timesteps")
+DEFAULT_CFG = 4
+_DIMS_TXT = "hidden 5376, 56x128 heads, ffn 14336, per-row timesteps"
+WORKLOADS = {
+    2: ("full-width MiniMax-H3 block, S=8192 packed rows (512 text | 6144 video (6,32,32) | "
+        "1536 audio), no padding, " + _DIMS_TXT),
+    3: ("full-width MiniMax-H3 block, S=16384 packed rows (1024 text | 12288 video (12,32,32) | "
+        "2560 audio | 512 padding rows in 4 runs, own attention document), " + _DIMS_TXT),
+    4: ("full-width MiniMax-H3 block, S=32768 packed rows (512 text | 30720 video (30,32,32) | "
+        "1536 audio), no padding, " + _DIMS_TXT),
+}
+MASKED_CFG = 3
 KERNELS = ["norm_modulate_1", "qkv_rope", "attention", "out_residual", "norm_modulate_2",
            "ffn_up", "ffn_down_residual"]
 
@@ -92,17 +106,19 @@ def block_flops(dims, V):
 KERNEL_SOURCES = {"norm_modulate_1": "norm.cu", "qkv_rope": "gemm.cu", "attention": "attention.cu",
                   "out_residual": "gemm.cu", "norm_modulate_2": "norm.cu", "ffn_up": "gemm.cu",
                   "ffn_down_residual": "gemm.cu"}
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_config2.txt")
+def traffic_file(cfg):
+    return os.path.join(ROOT, "profiles", f"dram_traffic_config{cfg}.txt")
 
 
-def measured_traffic(kernel):
+def measured_traffic(kernel, cfg=DEFAULT_CFG):
     """dram__bytes_read.sum + dram__bytes_write.sum per launch of `kernel` from the
-    committed ncu summary, or None if none was recorded for the current source."""
+    committed ncu summary of this workload, or None if none was recorded for the
+    kernel's current source."""
     src = os.path.join(ROOT, "audio_generation_b200", "csrc", KERNEL_SOURCES[kernel])
     try:
         with open(src, "rb") as f:
             digest = hashlib.sha256(f.read()).hexdigest()
-        with open(TRAFFIC_FILE) as f:
+        with open(traffic_file(cfg)) as f:
             lines = f.read().splitlines()
     except OSError:
         return None
@@ -214,59 +230,90 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle timing
 
-def oracle_sample(rows: int = 512):
-    """Time the oracle on the first ``rows`` text-like rows as a packed sequence of
-    their own; report rows/s scaled to the full workload's per-row work."""
-    from oracle import h3_oracle as O  # CPU baseline only
-    dims = FULL_DIMS
-    w = block_weights(dims, CFG, 0)
-    L = make_layout([("text", 0, rows)], seed=[CFG])
-    x = O.bf16_to_f64(activations(dims, CFG, rows))
-    pw = prologue_weights(dims, CFG)
-    t0 = time.perf_counter()
-    tm = O.timestep_modulation(L.timestep, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim,
-                               dims.hidden)
-    t1 = time.perf_counter()
-    O.block_forward(x, w, L, tm, dims)
-    t2 = time.perf_counter()
-    full_S = config_layout(CFG).S
-    per_row_sample = block_flops(dims, rows) / rows
-    per_row_full = block_flops(dims, full_S) / full_S
-    rate = rows / (t2 - t1) * (per_row_sample / per_row_full)
+def _cores():
     try:
-        cores = len(os.sched_getaffinity(0))
+        return len(os.sched_getaffinity(0))
     except AttributeError:
-        cores = os.cpu_count() or 1
-    return {
-        "value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
-        "sample": (f"float64 NumPy oracle block forward on {rows} packed rows as their own "
-                   f"sequence ({t2 - t1:.2f} s; prologue {t1 - t0:.2f} s not counted), rows/s "
-                   f"scaled by per-row work {per_row_sample / 1e6:.0f} / "
-                   f"{per_row_full / 1e6:.0f} MFLOP to the {full_S}-row workload"),
-    }
+        return os.cpu_count() or 1
+
+
+class OracleSampler:
+    """Bounded samples of one block forward of a workload on the CPU oracle.
+
+    Set-up (untimed): the workload's weights and inputs, and the keys and values
+    of every row of the sequence. A sample (timed) runs ``rows`` query rows
+    through the whole float64 block: their modulation, their own q, k and v,
+    attention over all S keys, the output projection, the FFN and both
+    residuals. Every row of the block costs the same, and the set-up's keys and
+    values are the other rows' share of the work, so rows / sample time
+    estimates the block's rows/s on the whole sequence.
+    """
+
+    def __init__(self, cfg):
+        from oracle import h3_oracle as O  # CPU baseline only
+        self.O = O
+        self.cfg = cfg
+        t0 = time.perf_counter()
+        self.dims = dims = FULL_DIMS
+        self.L = L = config_layout(cfg)
+        self.w = block_weights(dims, cfg, 0)
+        pw = prologue_weights(dims, cfg)
+        self.x = O.bf16_to_f64(activations(dims, cfg, L.S)[0])
+
+        def tmod_rows(ti, n_chunks):
+            return O.timestep_modulation(L.timestep[ti], pw.w_t1, pw.w_t2,
+                                         pw.w_proj[:n_chunks * dims.hidden], dims.freq_dim,
+                                         dims.hidden).reshape(len(ti), n_chunks, dims.hidden)
+
+        self.tmod_rows = tmod_rows
+        self.K, self.V = O.key_value_rows(self.x, self.w, L, tmod_rows, dims)
+        self.setup_s = time.perf_counter() - t0
+        self.rng = np.random.default_rng([cfg, 31337])
+
+    def sample(self, rows):
+        r = np.sort(self.rng.choice(self.L.S, size=rows, replace=False))
+        t0 = time.perf_counter()
+        self.O.query_rows(self.x, self.w, self.L, self.tmod_rows, self.dims, r, self.K, self.V)
+        return time.perf_counter() - t0
+
+    def describe(self, rows, n, secs):
+        return (f"float64 NumPy oracle block forward of {rows} random query rows per sample "
+                f"({n} samples, {secs:.2f} s each on average) over the {self.L.S}-row config-"
+                f"{self.cfg} sequence, keys and values of all rows formed beforehand "
+                f"({self.setup_s:.1f} s set-up, not counted)")
+
+
+def oracle_baseline(cfg, rows, samples):
+    """cpu_baseline: a few timed oracle samples of the bench's workload."""
+    smp = OracleSampler(cfg)
+    smp.sample(max(8, rows // 8))  # untimed warm-up (BLAS threads, caches)
+    times = [smp.sample(rows) for _ in range(samples)]
+    sec = statistics.median(times)
+    return {"value": rows / sec, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": smp.describe(rows, samples, sum(times) / len(times))}
 
 
 def run_reference(args, world, rank):
-    """The oracle as the reference arm: each step is one bounded CPU sample of the
-    workload; the run is time-boxed so that it ends within a few minutes."""
+    """The oracle as the reference arm: every step is one bounded CPU sample of
+    the workload (``--ref-rows`` query rows through the float64 block)."""
     if rank != 0:
         return 0
-    per = []
-    oracle_sample(args.ref_rows)  # one untimed warm-up sample (BLAS threads, caches)
-    t0 = time.perf_counter()
-    for _ in range(max(1, args.steps)):
-        per.append(oracle_sample(args.ref_rows))
-        if time.perf_counter() - t0 > args.ref_budget_s:
-            break
-    val = statistics.median(p["value"] for p in per)
-    base = per[0]
+    cfg = args.workload
+    smp = OracleSampler(cfg)
+    for _ in range(args.warmup):
+        smp.sample(args.ref_rows)
+    times = [smp.sample(args.ref_rows) for _ in range(args.steps)]
+    total = sum(times)
+    val = args.ref_rows * len(times) / total
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "samples_run": len(per),
-        "ms_per_step": config_layout(CFG).S / val * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / len(times) * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "S": config_layout(CFG).S, "B": 1},
-        "cpu_baseline": dict(base, value=val),
+        "config": {"workload": WORKLOADS[cfg], "S": config_layout(cfg).S, "B": 1,
+                   "step": f"{args.ref_rows} query rows of the block (bounded sample)"},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                         "sample": smp.describe(args.ref_rows, len(times), total / len(times))},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -288,7 +335,8 @@ def run_gpu(args, world, rank, local):
     torch.cuda.set_device(device)
     dims = FULL_DIMS
     d = h3.make_dims(dims)
-    L = config_layout(CFG)
+    cfg = args.workload
+    L = config_layout(cfg)
     S, V, B = L.S, L.n_valid, 1
 
     def to_dev_bits(a):
@@ -301,8 +349,8 @@ def run_gpu(args, world, rank, local):
     def to_dev_i32(a):
         return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
 
-    w = block_weights(dims, CFG, 0)
-    pw = prologue_weights(dims, CFG)
+    w = block_weights(dims, cfg, 0)
+    pw = prologue_weights(dims, cfg)
     wd = {k: to_dev_bits(getattr(w, k)) for k in ("w_qkv", "q_norm", "k_norm", "w_o", "w13", "w2")}
     wd["ada_table"] = to_dev_f32(w.ada_table)
     cw = h3.make_block_weights(wd["w_qkv"], wd["q_norm"], wd["k_norm"], wd["w_o"], wd["w13"],
@@ -317,7 +365,7 @@ def run_gpu(args, world, rank, local):
     h3.h3_timestep_modulation(d, L.n_t, to_dev_f32(L.timestep), to_dev_f32(pw.w_t1),
                               to_dev_f32(pw.w_t2), to_dev_f32(pw.w_proj), tmod, tws, tws_b)
     del tws
-    x_host = torch.from_numpy(activations(dims, CFG, S, B).view(np.int16)).view(
+    x_host = torch.from_numpy(activations(dims, cfg, S, B).view(np.int16)).view(
         torch.bfloat16).pin_memory()
     x = x_host.to(device)
     ws_b = h3.h3_workspace_size(d, B, S)
@@ -452,30 +500,34 @@ def run_gpu(args, world, rank, local):
                           "frac_of_peak": round(amt / t / 1e9 / peaks["hbm_gbs"], 3)}
     flops = block_flops(dims, V)
     clocks = clk.summary()
+    del hbuf, q, k, v, o, gbuf
+    masked = None if args.no_masked else masked_attention(h3, d, dims, device, stream, peaks)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded random-init weights and activations)",
-        "config": {"workload": WORKLOAD, "S": S, "B": B, "valid_rows": V,
-                   "l2": "inputs larger than L2 (770 MB of block weights + 1 GB tmod per step)",
+        "config": {"workload": WORKLOADS[cfg], "S": S, "B": B, "valid_rows": V,
+                   "l2": (f"inputs larger than L2 (770 MB of block weights + "
+                          f"{L.n_t * 6 * dims.hidden * 4 / 2**30:.1f} GiB tmod per step)"),
                    "parallelism": f"replicas x{world}, no collective on the data path"},
         "tflops": flops / (ms_per_step * 1e-3) / 1e12,
         "frac_of_peak": flops / (ms_per_step * 1e-3) / 1e12 / tc_peak,
         "frac_of_burst_peak": flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "peak_source": peaks["source"],
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
-                     "unit": unit, "frac": achieved / peak, "traffic": measured_traffic(dom),
+                     "unit": unit, "frac": achieved / peak, "traffic": measured_traffic(dom, cfg),
                      "peak_kind": peak_kind if bound == "tensor" else "copy",
                      "algorithmic_bytes": kernel_bytes(dims, V)[dom]},
         "kernels": kernels,
+        "attention_masked": masked,
         "e2e": {"value": world * B * S / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
         "gpu_launches": len(launches) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample(args.ref_rows)
+        line["cpu_baseline"] = oracle_baseline(cfg, args.ref_rows, 3)
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
@@ -483,6 +535,45 @@ def run_gpu(args, world, rank, local):
         dist.destroy_process_group()
     layout.close()
     return 0
+
+
+def masked_attention(h3, d, dims, device, stream, peaks, reps=10):
+    """The attention kernel alone on the padded 16384-row layout (512 padding
+    rows in four runs; two runs straddle a 128-row tile, so two tiles need the
+    per-key mask and two are skipped whole). Q, K and V are seeded N(0, 1) bf16
+    rows, the scale of q and k after the per-head RMSNorm. Reports the kernel's
+    mean time and TFLOP/s over the valid work, 4 NH D V^2 for the V valid rows
+    (the padding document is not counted)."""
+    import torch
+    L = config_layout(MASKED_CFG)
+    S, V = L.S, L.n_valid
+    to_i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+    pos = torch.from_numpy(np.ascontiguousarray(L.pos, dtype=np.float32)).to(device)
+    layout = h3.h3_layout_prepare(d, S, L.n_t, pos, to_i32(L.tags), to_i32(L.t_idx),
+                                  to_i32(L.video_idx), to_i32(L.audio_idx), to_i32(L.text_idx))
+    g = torch.Generator(device=device)
+    g.manual_seed(3003)
+    shape = (1, dims.heads, S, dims.head_dim)
+    q, k, v = (torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(
+        torch.bfloat16) for _ in range(3))
+    o = torch.empty((1, S, dims.attn_width), dtype=torch.bfloat16, device=device)
+    for _ in range(3):
+        h3.h3_attention(d, layout, 1, q, k, v, o, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(reps):
+        h3.h3_attention(d, layout, 1, q, k, v, o, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    if h3.h3_layout_error(layout) != h3.H3_OK:
+        raise RuntimeError("device error word set during the masked attention run")
+    layout.close()
+    ms = e0.elapsed_time(e1) / reps
+    tf = 4.0 * dims.heads * dims.head_dim * float(V) ** 2 / (ms * 1e-3) / 1e12
+    return {"workload": WORKLOADS[MASKED_CFG], "S": S, "valid_rows": V, "launches": reps,
+            "ms": round(ms, 4), "tflops_valid": round(tf, 1),
+            "frac_of_peak": round(tf / peaks["bf16_tflops"], 3), "peak_kind": "burst"}
 
 
 STACK_CFG = 5
@@ -587,14 +678,16 @@ def run_stack(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--ref-rows", type=int, default=512,
-                    help="rows of the oracle's bounded CPU sample")
-    ap.add_argument("--ref-budget-s", type=float, default=150.0,
-                    help="time box of the reference arm's timed samples")
+    ap.add_argument("--workload", type=int, choices=sorted(WORKLOADS), default=DEFAULT_CFG,
+                    help="single-block workload (4: 32768 rows; 3: 16384 padded; 2: 8192)")
+    ap.add_argument("--ref-rows", type=int, default=256,
+                    help="query rows per bounded oracle sample (one reference step)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-masked", action="store_true",
+                    help="skip the masked-attention measurement on the padded layout")
     ap.add_argument("--stack", action="store_true",
                     help="time the 50-block stack forward instead (one GPU, own JSON line)")
     args = ap.parse_args(argv)

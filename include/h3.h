@@ -31,7 +31,11 @@
  *  - Alignment: every device pointer must be 16-byte aligned.
  *  - Shapes: head_dim == 128; hidden % 256 == 0 and <= 6144; heads even;
  *    ffn % 128 == 0; rope_freq_dim == 16; freq_dim, time_hidden and
- *    time_embed_dim % 4 == 0. S (rows) is arbitrary >= 0.
+ *    time_embed_dim % 4 == 0. S (rows) is any value in [0, 524288] (the
+ *    attention kernel keeps the list of 128-row key tiles it visits in shared
+ *    memory); h3_layout_prepare returns H3_ERR_SHAPE for a larger S. B (batch
+ *    elements) is at most 65535 with B * S < 2^31; the batched calls return
+ *    H3_ERR_SHAPE beyond.
  *  - Batch: B >= 1 elements share one layout; each element is its own attention
  *    document set (the page's "pure replication axis").
  *  - Asynchronous failures: every wait inside a kernel is bounded (about 2 s).
@@ -180,11 +184,19 @@ H3_API h3_status h3_unpack_rows(h3_layout_t layout, int B, int row_elems, const 
  * From 65 timesteps on (when the widths allow) the three GEMMs run on the
  * tensor cores over three-way bf16 splits of both fp32 operands, whose copies
  * live in ws: the workspace then also holds, for the largest GEMM, n_t x 6K
- * and N x 6K bf16 values (about 1.3 GB at n_t = 8192 and the full widths). */
+ * and N x 6K bf16 values (about 1.3 GB at n_t = 8192 and the full widths).
+ * The split form's GEMMs have bounded waits like every kernel here; one that
+ * runs out records a timeout in a library-owned error word (one per GPU),
+ * which h3_timestep_error reads. */
 H3_API size_t h3_timestep_workspace_size(const h3_dims* dims, int n_t);
 H3_API h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const float* t, const float* w_t1,
                                  const float* w_t2, const float* w_proj, float* tmod, void* ws,
                                  size_t ws_bytes, h3_stream_t stream);
+
+/* Read and clear the error word of h3_timestep_modulation's split form on the
+ * current device (synchronises the device): H3_OK, or H3_ERR_TIMEOUT if one of
+ * its bounded in-kernel waits ran out since the last read. */
+H3_API h3_status h3_timestep_error(void);
 
 /* Same result as h3_timestep_modulation, for callers that cannot allocate device
  * memory (a serving loop whose device memory is reserved up front by its own
@@ -197,7 +209,10 @@ H3_API h3_status h3_timestep_modulation(const h3_dims* dims, int n_t, const floa
  * larger n_t returns H3_ERR_WORKSPACE before any work is queued. All calls on a device share the array: calls whose work
  * overlaps on the GPU race (order them on one stream or with events). Nothing in
  * the array needs to start at zero. The first call on a device looks up the
- * array's address; make it before any stream capture. */
+ * array's address; make it before any stream capture. The address is looked
+ * up again if the device's context has been replaced since (after a
+ * cudaDeviceReset). Arguments are checked like h3_timestep_modulation's: the
+ * same bad input gives the same status. */
 H3_API h3_status h3_timestep_modulation_noalloc(const h3_dims* dims, int n_t, const float* t,
                                                 const float* w_t1, const float* w_t2,
                                                 const float* w_proj, float* tmod,

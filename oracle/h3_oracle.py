@@ -283,21 +283,16 @@ def block_forward(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
     return out
 
 
-def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable, dims, rows: np.ndarray,
-                       chunk: int = 2048) -> np.ndarray:
-    """The same block evaluated only at the query rows ``rows`` (B = 1).
-
-    Keys and values are needed for every row, so they are formed for all rows
-    in row chunks (each row's k and v depend on that row alone).
-    ``tmod_rows(t_idx, n_chunks)`` returns the first ``n_chunks`` modulation
-    chunks of tmod for those timestep indices, [n, n_chunks, H]: the key/value
-    pass asks only for (shift1, scale1), so a caller with one timestep per row
-    never forms the whole tmod.
-    """
+def key_value_rows(x: np.ndarray, w, layout, tmod_rows: Callable, dims,
+                   chunk: int = 2048) -> Tuple[np.ndarray, np.ndarray]:
+    """k, v [S, NH, D] of every row of one sequence (B = 1), in row chunks (each
+    row's k and v depend on that row alone). ``tmod_rows(t_idx, n_chunks)``
+    returns the first ``n_chunks`` modulation chunks of tmod for those timestep
+    indices, [n, n_chunks, H]; this pass asks only for (shift1, scale1), so a
+    caller with one timestep per row never forms the whole tmod."""
     x = np.asarray(x, F)
     S = x.shape[0]
     tags = np.asarray(layout.tags)
-    pad = tags < 0
     NH, D = dims.heads, dims.head_dim
     K = np.empty((S, NH, D), F)
     V = np.empty((S, NH, D), F)
@@ -312,6 +307,19 @@ def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable, dims, rows
             m[vv] = table[tg[vv], :2] + tmod_rows(t_idx[r0:r1][vv], 2)
         _, K[r0:r1], V[r0:r1] = _pre_attention(x[r0:r1], m, layout.pos[r0:r1], w, dims,
                                                False, need_q=False)
+    return K, V
+
+
+def query_rows(x: np.ndarray, w, layout, tmod_rows: Callable, dims, rows: np.ndarray,
+               K: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """The block's output at the query rows ``rows`` (B = 1), given k and v of
+    every row (from ``key_value_rows``). The rows' own q, k and v are formed
+    here from their inputs, as in the block."""
+    x = np.asarray(x, F)
+    tags = np.asarray(layout.tags)
+    pad = tags < 0
+    table = np.asarray(w.ada_table, F)
+    t_idx = np.asarray(layout.t_idx)
     rows = np.asarray(rows)
     tg = tags[rows]
     m = np.zeros((rows.shape[0], 6, dims.hidden), F)
@@ -322,6 +330,18 @@ def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable, dims, rows
     o = attention(q, pad[rows], K, V, pad)
     y = _post_attention(x[rows], o, m, w, dims, False)
     return np.where(pad[rows][:, None], x[rows], y)
+
+
+def block_forward_rows(x: np.ndarray, w, layout, tmod_rows: Callable, dims, rows: np.ndarray,
+                       chunk: int = 2048) -> np.ndarray:
+    """The same block evaluated only at the query rows ``rows`` (B = 1).
+
+    Keys and values are needed for every row, so they are formed for all rows
+    first (``key_value_rows``), then the block runs at the query rows
+    (``query_rows``).
+    """
+    K, V = key_value_rows(x, w, layout, tmod_rows, dims, chunk)
+    return query_rows(x, w, layout, tmod_rows, dims, rows, K, V)
 
 
 def stack_forward(x: np.ndarray, weights_for_block: Callable[[int], object], n_blocks: int,

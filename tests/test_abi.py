@@ -152,3 +152,41 @@ def test_product_never_imports_the_oracle_and_vice_versa():
     assert not any(m.split(".")[0] in ("audio_generation_b200",) for m in _imports(os.path.join(ROOT, "oracle")))
     assert not any(m.split(".")[0] in ("audio_generation_b200", "oracle")
                    for m in _imports(os.path.join(ROOT, "workloads")))
+
+
+def test_row_limit_is_rejected_before_any_launch():
+    """S above 524288 (128 x 4096 key tiles, the attention kernel's shared-memory
+    key-tile list) is refused by h3_layout_prepare with H3_ERR_SHAPE; the check
+    comes before any device call (the pointers here are not device memory)."""
+    L = h3.lib()
+    d = h3.make_dims(FULL_DIMS)
+    out = ctypes.c_void_p()
+    fake = 1 << 20  # never dereferenced: the shape check comes first
+    for S, want in ((524289, h3.H3_ERR_SHAPE), (1 << 30, h3.H3_ERR_SHAPE)):
+        desc = h3.h3_layout_desc(S=S, n_t=1, pos=fake, tags=fake, t_idx=fake)
+        assert L.h3_layout_prepare(ctypes.byref(d), ctypes.byref(desc), None,
+                                   ctypes.byref(out)) == want
+        assert out.value is None
+
+
+def test_noalloc_and_workspace_prologue_check_arguments_alike():
+    """The no-allocation prologue returns the same status as the workspace form
+    for the same bad input, including n_t = 0 (nothing to compute)."""
+    L = h3.lib()
+    bad_eps = dict(FULL_DIMS.__dict__, norm_eps=0.0)
+    bad_shape = dict(FULL_DIMS.__dict__, hidden=500)
+    for kw, want in ((bad_eps, h3.H3_ERR_ARG), (bad_shape, h3.H3_ERR_SHAPE)):
+        d = h3.make_dims(Dims(**kw))
+        for n_t in (0, 3):
+            a = L.h3_timestep_modulation(ctypes.byref(d), n_t, None, None, None, None, None, None,
+                                         0, None)
+            b = L.h3_timestep_modulation_noalloc(ctypes.byref(d), n_t, None, None, None, None,
+                                                 None, None)
+            assert a == b == want, (kw, n_t, a, b)
+    d = h3.make_dims(FULL_DIMS)
+    assert L.h3_timestep_modulation(ctypes.byref(d), -1, None, None, None, None, None, None, 0,
+                                    None) == h3.H3_ERR_ARG
+    assert L.h3_timestep_modulation_noalloc(ctypes.byref(d), -1, None, None, None, None, None,
+                                            None) == h3.H3_ERR_ARG
+    assert L.h3_timestep_modulation_noalloc(ctypes.byref(d), 0, None, None, None, None, None,
+                                            None) == h3.H3_OK

@@ -62,20 +62,23 @@ def test_work_counts_match_the_stated_flops():
 
 
 def test_recorded_traffic_is_used_only_for_the_recorded_source(tmp_path, monkeypatch):
-    """roofline.traffic comes from the committed ncu summary only while the
-    kernel's source file still hashes to the recorded SHA-256."""
+    """roofline.traffic comes from the committed ncu summary of the bench's
+    workload, and only while the kernel's source file still hashes to the
+    recorded SHA-256."""
     import hashlib
     src = tmp_path / "k.cu"
     src.write_text("// a kernel\n")
     digest = hashlib.sha256(src.read_bytes()).hexdigest()
-    rec = tmp_path / "traffic.txt"
+    (tmp_path / "profiles").mkdir()
+    rec = tmp_path / "profiles" / "dram_traffic_config4.txt"
     rec.write_text(f"# comment line\nattention {digest} 123456\n")
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setitem(bench.KERNEL_SOURCES, "attention", "k.cu")
     (tmp_path / "audio_generation_b200" / "csrc").mkdir(parents=True)
     (tmp_path / "audio_generation_b200" / "csrc" / "k.cu").write_bytes(src.read_bytes())
     assert bench.measured_traffic("attention") == 123456.0
+    assert bench.measured_traffic("attention", 4) == 123456.0
+    assert bench.measured_traffic("attention", 3) is None  # no record for that workload
     (tmp_path / "audio_generation_b200" / "csrc" / "k.cu").write_text("// changed\n")
     assert bench.measured_traffic("attention") is None
 

@@ -587,3 +587,124 @@ def test_config_layouts_row_counts():
     L5 = config_layout(5)
     assert L5.n_t == 2 and L5.timestep[0] == 0.0
     assert set(np.unique(L5.t_idx).tolist()) == {0, 1}
+
+
+# ---------------------------------------------------------------- prologue worked by hand
+
+def test_timestep_modulation_worked_by_hand():
+    """A tiny prologue worked out by hand: freq_dim 4 (two frequencies,
+    f_0 = 1 and f_1 = (10^4)^(-1/2) = 0.01), time_hidden 2, time_embed_dim 2,
+    hidden 2 (six chunks of two), timesteps 0 and 0.5.
+
+    W_t1 = [[1, 0, 0, 0], [0, 0, 2, 100]] reads cos(t), then 2 sin(t) + 100 sin(0.01 t);
+    W_t2 = [[1, -1], [-2, 0]];  W_proj row (2c + j) = [c + 1, (-1)^j (j + 1) / 2].
+
+    t = 0:   sinusoid [cos 0, cos 0, sin 0, sin 0] = [1, 1, 0, 0]
+             W_t1 -> [1, 0];  SiLU(1) = 1 / (1 + e^-1) = 0.7310585786, SiLU(0) = 0
+             W_t2 -> temb = [0.7310585786, -1.4621171573]
+             SiLU -> [0.4934919753, -0.2750881685]
+             chunk c, column j = (c + 1) 0.4934919753 + (-1)^j (j + 1)/2 (-0.2750881685)
+               c = 0: [0.3559478910, 0.7685801438] ... c = 5: [2.8234077675, 3.2360400202]
+    t = 0.5: sinusoid [cos .5, cos .005, sin .5, sin .005]
+               = [0.8775825619, 0.9999875000, 0.4794255386, 0.0049999792]
+             W_t1 -> [0.8775825619, 0.9588510772 + 0.4999979167 = 1.4588489939]
+             SiLU -> [0.6198550086, 1.1836467133]
+             W_t2 -> temb = [-0.5637917047, -1.2397100173]
+             SiLU -> [-0.2044706686, -0.2782981200]
+               c = 0: [-0.3436197285, 0.0738274514] ... c = 5: [-1.3659730714, -0.9485258914]
+
+    A dropped or moved SiLU, swapped sin/cos halves, the frequency divisor
+    freq_dim instead of freq_dim / 2 (f_1 = 0.1), or a transposed chunk
+    reshape each changes these values far beyond the tolerance.
+    """
+    w_t1 = np.array([[1, 0, 0, 0], [0, 0, 2, 100]], F)
+    w_t2 = np.array([[1, -1], [-2, 0]], F)
+    w_proj = np.array([[c + 1, (-1) ** j * (j + 1) / 2] for c in range(6) for j in range(2)], F)
+    got = O.timestep_modulation(np.array([0.0, 0.5]), w_t1, w_t2, w_proj, 4, 2)
+    b0 = (0.49349197528601374, -0.2750881684806041)
+    b1 = (-0.20447066856192508, -0.278298119967226)
+    want = np.array([[[(c + 1) * b[0] + (-1) ** j * (j + 1) / 2 * b[1] for j in range(2)]
+                      for c in range(6)] for b in (b0, b1)])
+    assert got.shape == (2, 6, 2)
+    np.testing.assert_allclose(got, want, rtol=1e-9, atol=0)
+    # the first and last chunks, as listed above
+    np.testing.assert_allclose(got[0, 0], [0.3559478910, 0.7685801438], atol=1e-9)
+    np.testing.assert_allclose(got[0, 5], [2.8234077675, 3.2360400202], atol=1e-9)
+    np.testing.assert_allclose(got[1, 0], [-0.3436197285, 0.0738274514], atol=1e-9)
+    np.testing.assert_allclose(got[1, 5], [-1.3659730714, -0.9485258914], atol=1e-9)
+
+
+# ---------------------------------------------------------------- bf16 storage emulation
+
+# The device stores these activations as bf16, in this order, in one block:
+# h (norm1 output), q, k, v (after QK-norm and RoPE), P of each head before
+# P.V, o, x1, h2, g and x2. The emulation must round at exactly these points.
+def test_emulation_rounds_at_the_device_storage_points():
+    d = SMALL
+    L = make_layout([("text", 0, 20), ("pad", 5), ("video", (2, 2, 4), 0, 2), ("audio", 0, 7)],
+                    seed=[3])
+    S, H, NH, D, Fd = L.S, d.hidden, d.heads, d.head_dim, d.ffn
+    w = _weights_big_gates(d, 4)
+    tmod = _tmod_random(L.n_t, H, 5)
+    x = O.bf16_to_f64(f32_to_bf16_bits(np.random.default_rng(6).standard_normal((1, S, H))))
+    seen = []
+    base = O.round_bf16
+
+    def spy(a):
+        seen.append(np.shape(a))
+        return base(a)
+
+    O.round_bf16 = spy
+    try:
+        O.block_forward(x, w, L, tmod, d, emulate=False)
+        assert seen == []
+        O.block_forward(x, w, L, tmod, d, emulate=True)
+    finally:
+        O.round_bf16 = base
+    want = ([(S, H), (S, NH, D), (S, NH, D), (S, NH, D)] + [(S, S)] * NH +
+            [(S, NH * D), (S, H), (S, H), (S, Fd), (S, H)])
+    assert seen == want
+
+
+def test_emulated_attention_rounds_p_but_sums_unrounded_p():
+    """One query, two keys, D = 1, so s = [0, ln p1] and the weights are
+    [1, p1] with p1 = 0.50244140625 = 0.5 (1 + 2^-8 + 2^-10). bf16 keeps 7
+    fraction bits: 1.0048828125 lies above the midpoint 1.00390625 between 1
+    and 1.0078125, so P rounds to [1, 0.50390625]; the row sum l is taken
+    from the unrounded weights, l = 1.50244140625 (the kernel adds fp32 p).
+
+    (a) v = [0, v1] with the exact output p1 v1 / l = 1.00341796875, just below
+        the midpoint 1.00390625: unrounded P would store o = 1.0; rounded P
+        gives 1.00341796875 * 0.50390625 / 0.50244140625 = 1.006343..., stored
+        as 1.0078125.
+    (b) the rounded-P output p1r v1 / l = 1.00439453125, just above the
+        midpoint: stored as 1.0078125; dividing by the sum of the rounded
+        weights (1.50390625) instead would give 1.003417..., stored as 1.0.
+    """
+    p1, p1r, l = 0.50244140625, 0.50390625, 1.50244140625
+    q = np.ones((1, 1, 1))
+    k = np.array([0.0, math.log(p1)]).reshape(2, 1, 1)
+    doc_q, doc_k = np.zeros(1, bool), np.zeros(2, bool)
+    v1a = 1.00341796875 * l / p1
+    va = np.array([0.0, v1a]).reshape(2, 1, 1)
+    assert O.attention(q, doc_q, k, va, doc_k)[0, 0] == pytest.approx(1.00341796875, rel=1e-12)
+    assert O.attention(q, doc_q, k, va, doc_k, emulate=True)[0, 0] == 1.0078125
+    v1b = 1.00439453125 * l / p1r
+    vb = np.array([0.0, v1b]).reshape(2, 1, 1)
+    assert O.attention(q, doc_q, k, vb, doc_k, emulate=True)[0, 0] == 1.0078125
+    assert O.round_bf16(np.array(p1r * v1b / (1 + p1r)))[()] == 1.0
+
+
+def test_emulated_residual_rounds_after_the_add():
+    """x1 = bf16(x + gate * (o W_o^T)): with x = 1, gate = 1 and a branch of
+    2^-9 (exact in bf16), the sum 1.001953125 is below the midpoint 1.00390625
+    and is stored as 1.0; a branch of 3 * 2^-9 gives 1.005859375, stored as
+    1.0078125. Rounding the branch alone and adding it unrounded would keep
+    1.001953125."""
+    w_o = f32_to_bf16_bits(np.array([[2.0 ** -9]], np.float32))
+    x = np.ones((1, 1))
+    for o, want in ((1.0, 1.0), (3.0, 1.0078125)):
+        got = O.out_project_residual(x, np.array([[o]]), np.ones((1, 1)), w_o, emulate=True)
+        assert got[0, 0] == want
+    got = O.out_project_residual(x, np.array([[1.0]]), np.ones((1, 1)), w_o, emulate=False)
+    assert got[0, 0] == 1.001953125
