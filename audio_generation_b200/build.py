@@ -54,6 +54,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_fault_injection(out_path: str, verbose: bool = False) -> str:
+    """A test-only variant of the library (never the product build): bounded
+    waits limited to 50 ms and an extra entry point, h3_test_gemm_skip_loads,
+    that makes the GEMM producer issue no loads, so a test can make a wait run
+    out and check the status the library reports."""
+    nvcc = os.environ.get("NVCC", "nvcc")
+    tmp = out_path + ".tmp"
+    cmd = [nvcc] + NVCC_FLAGS + ["-DH3_FAULT_INJECTION", "-I", INCLUDE, "-o", tmp] + sources()
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out_path)
+    return out_path
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True)
     print(LIB)

@@ -186,10 +186,14 @@ h3_status h3_layout_prepare(const h3_dims* dims, const h3_layout_desc* desc, h3_
   const size_t sz_i = align256((size_t)S * 4), sz_pos = align256((size_t)S * 12),
                sz_rope = align256((size_t)S * kRopePairs * 8), sz_tc = align256(nt),
                sz_kv = align256(nt * 16);
-  const size_t total = 6 * sz_i /*tags t_idx src perm c_tags c_tidx*/ + sz_pos + 2 * sz_rope +
-                       2 * sz_tc + 2 * sz_kv + align256((size_t)desc->n_video * 4) +
+  const size_t n_tt = (desc->n_text + kTile - 1) / kTile;
+  const size_t sz_ti = align256((size_t)desc->n_text * 4),
+               sz_trope = align256((size_t)desc->n_text * kRopePairs * 8),
+               sz_ttc = align256(n_tt), sz_tkv = align256(n_tt * 16);
+  const size_t total = 7 * sz_i /*tags t_idx src perm c_tags c_tidx c_of_row*/ + sz_pos +
+                       2 * sz_rope + 2 * sz_tc + 2 * sz_kv + align256((size_t)desc->n_video * 4) +
                        align256((size_t)desc->n_audio * 4) + align256((size_t)desc->n_text * 4) +
-                       256 /*err*/;
+                       2 * sz_ti + sz_trope + sz_ttc + sz_tkv /*text view*/ + 256 /*err*/;
   if (cudaMalloc(&L->block, total) != cudaSuccess) {
     delete L;
     return H3_ERR_CUDA;
@@ -216,6 +220,13 @@ h3_status h3_layout_prepare(const h3_dims* dims, const h3_layout_desc* desc, h3_
   L->video_idx = reinterpret_cast<int32_t*>(take(align256((size_t)desc->n_video * 4)));
   L->audio_idx = reinterpret_cast<int32_t*>(take(align256((size_t)desc->n_audio * 4)));
   L->text_idx = reinterpret_cast<int32_t*>(take(align256((size_t)desc->n_text * 4)));
+  L->c_of_row = reinterpret_cast<int32_t*>(take(sz_i));
+  L->t_tags = reinterpret_cast<int32_t*>(take(sz_ti));
+  L->t_tidx = reinterpret_cast<int32_t*>(take(sz_ti));
+  L->t_rope = reinterpret_cast<float2*>(take(sz_trope));
+  L->t_tile_class = take(sz_ttc);
+  L->t_key_valid = reinterpret_cast<uint32_t*>(take(sz_tkv));
+  L->t_tiles = (int)n_tt;
   L->err = reinterpret_cast<int*>(take(256));
 
   h3_status rc = H3_OK;
@@ -489,6 +500,130 @@ h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* weights,
   for (int i = 0; i < n_blocks; ++i)
     H3_TRY(run_block(*dims, weights[i], L->compact_view(), tmod, w.xc, true, B, w, st));
   H3_CUDA(launch_permute_rows_convert(B, V, L->S, dims->hidden, L->perm, w.xc, x, false, st));
+  return H3_OK;
+}
+
+}  // extern "C"
+
+// ---- the denoiser around the stack ----
+
+namespace {
+
+h3_status check_io(const h3_dims* d, const h3_io_dims* io) {
+  if (!io) return H3_ERR_ARG;
+  if (!io_channels_supported(io->video_channels) || !io_channels_supported(io->audio_channels))
+    return H3_ERR_SHAPE;
+  if (io->text_dim <= 0 || io->text_dim % 64 != 0) return H3_ERR_SHAPE;
+  if (!(io->final_norm_eps > 0.f)) return H3_ERR_ARG;
+  (void)d;
+  return H3_OK;
+}
+
+// Parts of h3_forward's workspace, in order: the stack's block workspace (its
+// fp32 stream xc is the forward's residual stream), the refiner's fp32 text
+// stream, tmod, tmod_out, and the prologue's scratch.
+struct ForwardWs {
+  void* block;
+  float *text, *tmod, *tmod_out;
+  void* prologue;
+};
+
+size_t forward_parts(const h3_dims& d, const h3_layout* L, int B, ForwardWs* w, void* base) {
+  const size_t block_b = ws_parts(d, B, L->S, nullptr, nullptr);
+  const size_t text_b = align256((size_t)B * L->n_text * d.hidden * 4);
+  const size_t tmod_b = align256((size_t)L->n_t * 6 * d.hidden * 4);
+  const size_t tout_b = align256((size_t)L->n_t * 2 * d.hidden * 4);
+  const size_t pro_b = align256(timestep_workspace_bytes(d, L->n_t, true));
+  if (w) {
+    uint8_t* p = static_cast<uint8_t*>(base);
+    w->block = p;
+    w->text = reinterpret_cast<float*>(p + block_b);
+    w->tmod = reinterpret_cast<float*>(p + block_b + text_b);
+    w->tmod_out = reinterpret_cast<float*>(p + block_b + text_b + tmod_b);
+    w->prologue = p + block_b + text_b + tmod_b + tout_b;
+  }
+  return block_b + text_b + tmod_b + tout_b + pro_b;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t h3_forward_workspace_size(const h3_dims* dims, const h3_io_dims* io, h3_layout_t L,
+                                 int B) {
+  if (check_dims(dims) != H3_OK || check_io(dims, io) != H3_OK || check_batch(L, B) != H3_OK)
+    return 0;
+  return forward_parts(*dims, L, B, nullptr, nullptr);
+}
+
+h3_status h3_forward(const h3_dims* dims, const h3_io_dims* io, const h3_io_weights* iw,
+                     const h3_block_weights* refiner, int n_refiner,
+                     const h3_block_weights* blocks, int n_blocks, h3_layout_t L,
+                     const float* timestep, int B, const float* video, const float* audio,
+                     const void* text, float* video_out, float* audio_out, void* ws,
+                     size_t ws_bytes, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  H3_TRY(check_io(dims, io));
+  if (!L || !iw || n_refiner < 0 || n_blocks < 0 || (n_refiner > 0 && !refiner) ||
+      (n_blocks > 0 && !blocks) || !ws)
+    return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
+  if (L->n_t > 0 && !timestep) return H3_ERR_ARG;
+  if (!iw->w_t1 || !iw->w_t2 || !iw->w_proj || !iw->w_out || !iw->out_table)
+    return H3_ERR_ARG;
+  if (L->n_video && (!video || !video_out || !iw->w_patch_video || !iw->w_head_video))
+    return H3_ERR_ARG;
+  if (L->n_audio && (!audio || !audio_out || !iw->w_patch_audio || !iw->w_head_audio))
+    return H3_ERR_ARG;
+  if (L->n_text && (!text || !iw->w_text)) return H3_ERR_ARG;
+  for (int i = 0; i < n_refiner; ++i) H3_TRY(check_weights(&refiner[i]));
+  for (int i = 0; i < n_blocks; ++i) H3_TRY(check_weights(&blocks[i]));
+  const void* ptrs[] = {timestep, video, audio, text, video_out, audio_out, ws, iw->w_patch_video,
+                        iw->w_patch_audio, iw->w_text, iw->w_t1, iw->w_t2, iw->w_proj,
+                        iw->w_out, iw->out_table, iw->w_head_video, iw->w_head_audio};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return H3_ERR_ALIGN;
+  if (ws_bytes < forward_parts(*dims, L, B, nullptr, nullptr)) return H3_ERR_WORKSPACE;
+  if (B == 0) return H3_OK;
+  cudaStream_t st = as_stream(stream);
+  const h3_dims& d = *dims;
+  const int H = d.hidden, V = L->n_valid;
+  ForwardWs fw;
+  forward_parts(d, L, B, &fw, ws);
+  Workspace w, wt;
+  ws_parts(d, B, L->S, &w, fw.block);
+  ws_parts(d, B, L->n_text, &wt, fw.block);  // the refiner's scratch, below w.xc
+  float* xc = static_cast<float*>(w.xc);
+  // timestep MLP, the stack's shared AdaLN projection and norm_out's modulation
+  if (L->n_t > 0)
+    H3_CUDA(launch_timestep(d, L->n_t, timestep, iw->w_t1, iw->w_t2, iw->w_proj, fw.tmod,
+                            fw.prologue, true, st, iw->w_out, fw.tmod_out));
+  // input projections into the residual stream
+  H3_CUDA(launch_patch_project(B, L->n_video, H, V, io->video_channels, video, iw->w_patch_video,
+                               L->video_idx, L->c_of_row, xc, st));
+  H3_CUDA(launch_patch_project(B, L->n_audio, H, V, io->audio_channels, audio, iw->w_patch_audio,
+                               L->audio_idx, L->c_of_row, xc, st));
+  if (L->n_text > 0) {
+    // text projection (bf16 weights, fp32 out), the refiner blocks on the text
+    // rows alone, and the refiner's output norm into the residual stream
+    GemmEpiArgs ea;
+    ea.L.err = L->err;
+    ea.out = fw.text;
+    H3_CUDA(launch_gemm(EPI_F32, B * L->n_text, H, io->text_dim, text, iw->w_text, ea, st));
+    for (int i = 0; i < n_refiner; ++i)
+      H3_TRY(run_block(d, refiner[i], L->text_view(), fw.tmod, fw.text, true, B, wt, st));
+    H3_CUDA(launch_rows_layer_norm(B, L->n_text, H, V, io->final_norm_eps, fw.text, L->text_idx,
+                                   L->c_of_row, xc, st));
+  }
+  for (int i = 0; i < n_blocks; ++i)
+    H3_TRY(run_block(d, blocks[i], L->compact_view(), fw.tmod, xc, true, B, w, st));
+  // norm_out and the two heads, in the order of the index tensors
+  H3_CUDA(launch_out_head(B, L->n_video, H, V, io->video_channels, io->final_norm_eps, xc,
+                          L->video_idx, L->c_of_row, L->t_idx, iw->out_table, fw.tmod_out,
+                          iw->w_head_video, video_out, st));
+  H3_CUDA(launch_out_head(B, L->n_audio, H, V, io->audio_channels, io->final_norm_eps, xc,
+                          L->audio_idx, L->c_of_row, L->t_idx, iw->out_table + 2 * H,
+                          fw.tmod_out, iw->w_head_audio, audio_out, st));
   return H3_OK;
 }
 

@@ -24,8 +24,10 @@
 // guarantees PV_i(j) is complete: the softmax may then rescale O_i in place.
 // O is rescaled only when a row's running max grows by more than 2^8 (lazy
 // rescale), decided per warp because TMEM loads / stores are warp-collective.
-// exp2 runs on the MUFU for three quarters of the keys and as a polynomial on
-// the FMA pipe for the last quarter, to balance the two pipes.
+// exp2 runs on the MUFU for three quarters of the key pairs and as a
+// polynomial on the FMA pipe for every fourth pair, to keep both pipes busy.
+// P is handed to the MMA warp in two halves (keys 0..63, then 64..127), so the
+// first half of P V runs while the second half's exponentials are computed.
 //
 // Document mask: per 128-row tile the layout step records whether it is all
 // valid, all padding or mixed, plus a valid-row bitmask. Key tiles that are
@@ -56,8 +58,8 @@ constexpr int kMaxKeyTiles = kMaxRows / 128;  // the key-tile list below (S <= k
 constexpr int SMEM_BYTES = OFF_LIST + 2 * kMaxKeyTiles + 1024;
 
 struct Bars {
-  uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2],
-      o_final[2], drain;
+  uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_half[2],
+      p_full[2], o_final[2], drain;
 };
 
 
@@ -67,21 +69,17 @@ __device__ __forceinline__ float exp2_mufu(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe: split x = j + f with j = round(x) (adding 1.5 * 2^23
-// leaves the rounded integer in the low mantissa bits) and f in [-1/2, 1/2];
-// 2^f by a cubic fitted by least squares (relative error weighted) at 256
-// Chebyshev nodes of [-1/2, 1/2], max relative error 7.7e-5 wherever 2^x is a
-// normal float (x >= -125; bf16 keeps 3.9e-3); j is added to the exponent
-// field. Inputs below -126 are clamped; below -125 the result is off by less
-// than 2^-135 in absolute terms, negligible next to the row sum, which is >= 1.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.05508868396f, f, 0.24260404706f), f, 0.69327622652f), f,
-                       0.99992895126f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
+// 2^x on the FMA pipe, for two values at once: split x = j + f with
+// j = round(x) (adding 1.5 * 2^23 leaves the rounded integer in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic fitted by least squares
+// (relative error weighted) at 256 Chebyshev nodes of [-1/2, 1/2], max
+// relative error 7.7e-5 wherever 2^x is a normal float (x >= -125; bf16 keeps
+// 3.9e-3); j is added to the exponent field. Inputs below -126 are clamped;
+// below -125 the result is off by less than 2^-135 in absolute terms,
+// negligible next to the row sum, which is >= 1.
+constexpr float kExpC3 = 0.05508868396f, kExpC2 = 0.24260404706f, kExpC1 = 0.69327622652f,
+                kExpC0 = 0.99992895126f;
+constexpr float kRoundMagic = 12582912.f;  // 1.5 * 2^23
 
 // Packed fp32 pair arithmetic (one instruction for two lanes of work).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
@@ -102,6 +100,30 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& p0, float& p1) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = f2_add(xc, f2_pack(kRoundMagic, kRoundMagic));
+  const uint64_t jf = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));     // j, exact
+  const uint64_t f = f2_fma(jf, f2_pack(-1.f, -1.f), xc);                  // x - j, exact
+  uint64_t p = f2_fma(f2_pack(kExpC3, kExpC3), f, f2_pack(kExpC2, kExpC2));
+  p = f2_fma(p, f, f2_pack(kExpC1, kExpC1));
+  p = f2_fma(p, f, f2_pack(kExpC0, kExpC0));
+  float q0, q1, t0, t1;
+  f2_unpack(p, q0, q1);
+  f2_unpack(t, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// Which key pairs of a 64-key half take the FMA-pipe exp2: every kPolyEvery-th
+// pair, spread among the MUFU pairs so that both pipes work at the same time.
+#ifndef H3_ATTN_POLY_EVERY
+#define H3_ATTN_POLY_EVERY 4
+#endif
+constexpr int kPolyEvery = H3_ATTN_POLY_EVERY;
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
@@ -170,7 +192,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->p_half[i], 4);  // one arrival per softmax warp
+      mbar_init(&bars->p_full[i], 4);
       mbar_init(&bars->o_final[i], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -259,17 +282,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (i == 1) umma_commit_elect(&bars->k_empty[st]);
         return true;
       };
-      // O_i += P_i(j) V_j, P_i from TMEM columns [128 i, 128 i + 64)
+      // O_i += P_i(j) V_j, P_i from TMEM columns [128 i, 128 i + 64). Keys
+      // 0..63 (P columns [0, 32)) go as soon as the softmax has stored them,
+      // keys 64..127 when the rest of P is in.
       auto issue_pv = [&](int i, int j) -> bool {
         const int st = j & 1;
-        if (!wait_all(&bars->p_full[i], j & 1)) return false;
+        if (!wait_all(&bars->p_half[i], j & 1)) return false;
         if (i == 0 && !wait_all(&bars->v_full[st], (j >> 1) & 1)) return false;
         tc_fence_after();
         const uint32_t vl = v_lo + st * (TILE_BYTES >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < 4; ++kk) {
           umma_ts_w_elect(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, vl + kk * (2048 >> 4), hi,
                           idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (!wait_all(&bars->p_full[i], j & 1)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 4; kk < 8; ++kk) {
+          umma_ts_w_elect(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, vl + kk * (2048 >> 4), hi,
+                          idesc_pv, 1u);
         }
         if (i == 1) umma_commit_elect(&bars->v_empty[st]);
         if (j == n - 1) umma_commit_elect(&bars->o_final[i]);
@@ -358,8 +390,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         m_run = m_new;
       }
-      // P = 2^(s * scale - m): keys 0..95 on the MUFU, 96..127 on the FMA pipe;
-      // packed bf16 pairs overwrite S columns already held in registers.
+      // P = 2^(s * scale - m), written as packed bf16 pairs over S columns
+      // already held in registers: keys 0..63, then keys 64..127, each half
+      // signalled to the MMA warp as soon as it is stored (one arrival per warp,
+      // after the warp's stores are complete). Every kPolyEvery-th key pair
+      // takes the FMA-pipe exp2, the others the MUFU.
       const uint64_t negm2 = f2_pack(-m_run, -m_run);
       uint64_t sum2[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -369,27 +404,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int e = 0; e < 32; ++e) {
           const int key = 64 * h + 2 * e;
           const uint64_t x2 = f2_fma(f2_pack(sc[key], sc[key + 1]), scale2, negm2);
-          float x0, x1, p0, p1;
-          f2_unpack(x2, x0, x1);
-          if (key < 96) {
+          float p0, p1;
+          if (e % kPolyEvery == kPolyEvery - 1) {
+            exp2_poly2(x2, p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
             p0 = exp2_mufu(x0);
             p1 = exp2_mufu(x1);
-          } else {
-            p0 = exp2_poly(x0);
-            p1 = exp2_poly(x1);
           }
           sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st32(s_col + 32 * h, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(h == 0 ? &bars->p_half[i] : &bars->p_full[i]);
       }
       float a0, a1, b0, b1;
       f2_unpack(f2_add(sum2[0], sum2[1]), a0, a1);
       f2_unpack(f2_add(sum2[2], sum2[3]), b0, b1);
       l_run += (a0 + a1) + (b0 + b1);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[i]);
     }
     if (ok && j > 0)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final[i], 0, wc));

@@ -53,6 +53,12 @@ constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 192;
 
+#ifdef H3_FAULT_INJECTION
+// Test-only build: when set, the producer issues no loads, so the MMA warp's
+// bounded wait on the first stage runs out (nothing else sets that barrier).
+static __device__ int g_fault_skip_loads;
+#endif
+
 __device__ __forceinline__ void store_bf16x32(void* dst, const float* y) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -301,6 +307,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       uint32_t n = 0;
       bool ok = true;
+#ifdef H3_FAULT_INJECTION
+      if (*(volatile int*)&g_fault_skip_loads) ok = false;
+#endif
       for (int t = pair; t < T && ok; t += n_pairs) {
         int m0, n0;
         tile_coords<BN>(t, tiles_m, tiles_n, group_n, m0, n0);
@@ -458,3 +467,10 @@ cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void*
 }
 
 }  // namespace h3
+
+#ifdef H3_FAULT_INJECTION
+// Test-only build: turn the GEMM producer's load skipping on (1) or off (0).
+extern "C" __attribute__((visibility("default"))) int h3_test_gemm_skip_loads(int on) {
+  return cudaMemcpyToSymbol(h3::g_fault_skip_loads, &on, sizeof(int)) == cudaSuccess ? 0 : -1;
+}
+#endif

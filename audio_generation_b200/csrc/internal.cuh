@@ -53,6 +53,13 @@ struct h3_layout {
   uint8_t* c_tile_class = nullptr;
   uint32_t* c_key_valid = nullptr;
   int c_tiles = 0;
+  int32_t* c_of_row = nullptr;  // [S] compact position of each packed row, -1 for padding
+  // the text rows alone (text_idx order): the refiner's sequence
+  int32_t *t_tags = nullptr, *t_tidx = nullptr;
+  float2* t_rope = nullptr;
+  uint8_t* t_tile_class = nullptr;
+  uint32_t* t_key_valid = nullptr;
+  int t_tiles = 0;
   int* err = nullptr;
   std::vector<uint8_t> tile_class_host;
 
@@ -61,6 +68,10 @@ struct h3_layout {
   }
   h3::LayoutView compact_view() const {
     return h3::LayoutView{n_valid, c_tiles, c_tags, c_tidx, c_rope, c_tile_class, c_key_valid,
+                          err};
+  }
+  h3::LayoutView text_view() const {
+    return h3::LayoutView{n_text, t_tiles, t_tags, t_tidx, t_rope, t_tile_class, t_key_valid,
                           err};
   }
 };
@@ -96,9 +107,11 @@ cudaError_t launch_norm_modulate(const LayoutView& L, int B, int H, int chunk_sh
 // operands (allow_split = false forces the first form). Workspace bytes for
 // either form; ws must be 256-byte aligned.
 size_t timestep_workspace_bytes(const h3_dims& d, int n_t, bool allow_split);
+// With w_out (else null) it also writes tmod_out = W_out . SiLU(temb) [n_t, 2H].
 cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const float* w_t1,
                             const float* w_t2, const float* w_proj, float* tmod, void* ws,
-                            bool allow_split, cudaStream_t st);
+                            bool allow_split, cudaStream_t st, const float* w_out = nullptr,
+                            float* tmod_out = nullptr);
 
 // EPI_RESID_F32: gated residual on an fp32 residual stream (inside the stack).
 enum GemmEpilogue {
@@ -134,6 +147,24 @@ cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, 
                              const void* v, void* o, cudaStream_t st);
 
 int num_sms();
+
+// ---- the denoiser around the stack (denoiser.cu) ----
+// Latent / velocity row widths the projection and head kernels take.
+bool io_channels_supported(int C);
+// xc[b, c_of_row[idx[i]]] = W . lat[b, i] (fp32; lat [B, n, C], W [H, C]).
+cudaError_t launch_patch_project(int B, int n, int H, int V, int C, const float* lat,
+                                 const float* W, const int32_t* idx, const int32_t* c_of_row,
+                                 float* xc, cudaStream_t st);
+// xc[b, c_of_row[idx[i]]] = LayerNorm(src[b, i]) (no affine).
+cudaError_t launch_rows_layer_norm(int B, int n, int H, int V, float eps, const float* src,
+                                   const int32_t* idx, const int32_t* c_of_row, float* xc,
+                                   cudaStream_t st);
+// out[b, i] = W . (LN(x) (1 + scale) + shift), x = xc[b, c_of_row[idx[i]]],
+// (shift, scale) = table[0..1] + tmod_out[t_idx[idx[i]]][0..1] (fp32; W [C, H]).
+cudaError_t launch_out_head(int B, int n, int H, int V, int C, float eps, const float* xc,
+                            const int32_t* idx, const int32_t* c_of_row, const int32_t* t_idx,
+                            const float* table, const float* tmod_out, const float* W,
+                            float* out, cudaStream_t st);
 
 // Shape checks shared by the entry points (H3_OK or the status to return).
 h3_status check_dims(const h3_dims* d);

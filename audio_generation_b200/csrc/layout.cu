@@ -157,6 +157,13 @@ __global__ void k_compact_tables(int V, int c_tiles, const int32_t* __restrict__
   }
 }
 
+// c_of_row[perm[j]] = j for the V valid rows (the caller fills c_of_row with -1).
+__global__ void k_compact_position(int V, const int32_t* __restrict__ perm,
+                                   int32_t* __restrict__ c_of_row) {
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < V; j += gridDim.x * blockDim.x)
+    c_of_row[perm[j]] = j;
+}
+
 // ---- a1: packed-row gather / scatter, one warp per row, 16-byte vectors ----
 
 __global__ void k_pack(int B, int S, int vec_per_row, const int32_t* __restrict__ src_of_row,
@@ -292,6 +299,19 @@ cudaError_t launch_compact_tables(h3_layout* L, cudaStream_t st) {
   k_compact_tables<<<grid_for((long long)(V > 0 ? V : 1) * kRopePairs, 256), 256, 0, st>>>(
       V, L->c_tiles, L->perm, L->tags, L->t_idx, L->rope, L->c_tags, L->c_tidx, L->c_rope,
       L->c_tile_class, L->c_key_valid);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // The text rows as a sequence of their own, in text_idx order: the same
+  // gather over text_idx instead of the compaction order.
+  const int T = L->n_text;
+  k_compact_tables<<<grid_for((long long)(T > 0 ? T : 1) * kRopePairs, 256), 256, 0, st>>>(
+      T, L->t_tiles, L->text_idx, L->tags, L->t_idx, L->rope, L->t_tags, L->t_tidx, L->t_rope,
+      L->t_tile_class, L->t_key_valid);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (L->S > 0) {
+    if ((e = cudaMemsetAsync(L->c_of_row, 0xff, (size_t)L->S * 4, st)) != cudaSuccess) return e;
+    if (V > 0) k_compact_position<<<grid_for(V, 256), 256, 0, st>>>(V, L->perm, L->c_of_row);
+  }
   return cudaGetLastError();
 }
 

@@ -18,8 +18,14 @@
 
 namespace h3 {
 
+#ifdef H3_FAULT_INJECTION
+// Test-only build (never the product library): short waits, so that a test
+// can make one run out and check the reported status.
+constexpr unsigned long long kWaitLimitNs = 50000000ull;
+#else
 // ~2 s: far above any legitimate wait inside one launch of this library.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

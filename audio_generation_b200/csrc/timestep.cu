@@ -10,6 +10,8 @@
 //   h1    = W_t1 e
 //   temb  = W_t2 SiLU(h1)
 //   tmod  = W_proj SiLU(temb)          -> [n_t, 6, H]
+//   tmod_out = W_out SiLU(temb)        -> [n_t, 2, H] (norm_out's shift and scale,
+//                                         when the caller asks for it)
 //
 // Runs once per forward for the distinct timestep values. Two forms of the
 // three fp32 GEMMs:
@@ -211,7 +213,8 @@ size_t timestep_workspace_bytes(const h3_dims& d, int n_t, bool allow_split) {
 
 cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const float* w_t1,
                             const float* w_t2, const float* w_proj, float* tmod, void* ws,
-                            bool allow_split, cudaStream_t st) {
+                            bool allow_split, cudaStream_t st, const float* w_out,
+                            float* tmod_out) {
   if (n_t == 0) return cudaSuccess;
   float* e = static_cast<float*>(ws);               // [n_t, freq_dim]
   float* h1 = e + (size_t)n_t * d.freq_dim;          // [n_t, time_hidden]
@@ -229,6 +232,9 @@ cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const flo
     if ((err = skinny(n_t, d.time_embed_dim, d.time_hidden, h1, w_t2, temb, st)) != cudaSuccess)
       return err;
     if ((err = silu_inplace((size_t)n_t * d.time_embed_dim, temb, st)) != cudaSuccess) return err;
+    if (w_out && (err = skinny(n_t, 2 * d.hidden, d.time_embed_dim, temb, w_out, tmod_out, st)) !=
+                     cudaSuccess)
+      return err;
     return skinny(n_t, 6 * d.hidden, d.time_embed_dim, temb, w_proj, tmod, st);
   }
   // Split operands of one stage at a time, after the fp32 activations.
@@ -251,6 +257,9 @@ cudaError_t launch_timestep(const h3_dims& d, int n_t, const float* t, const flo
   };
   if ((err = gemm_stage(d.freq_dim, d.time_hidden, e, false, w_t1, h1)) != cudaSuccess) return err;
   if ((err = gemm_stage(d.time_hidden, d.time_embed_dim, h1, true, w_t2, temb)) != cudaSuccess)
+    return err;
+  if (w_out && (err = gemm_stage(d.time_embed_dim, 2 * d.hidden, temb, true, w_out, tmod_out)) !=
+                   cudaSuccess)
     return err;
   return gemm_stage(d.time_embed_dim, 6 * d.hidden, temb, true, w_proj, tmod);
 }

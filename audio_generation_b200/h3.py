@@ -55,6 +55,17 @@ class h3_block_weights(ctypes.Structure):
         "w_qkv", "q_norm", "k_norm", "w_o", "w13", "w2", "ada_table")]
 
 
+class h3_io_dims(ctypes.Structure):
+    _fields_ = [("video_channels", ctypes.c_int), ("audio_channels", ctypes.c_int),
+                ("text_dim", ctypes.c_int), ("final_norm_eps", ctypes.c_float)]
+
+
+class h3_io_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_patch_video", "w_patch_audio", "w_text", "w_t1", "w_t2", "w_proj", "w_out",
+        "out_table", "w_head_video", "w_head_audio")]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -85,6 +96,12 @@ _SIGNATURES = {
                                   _vp]),
     "h3_block_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _vp,
                               _vp, _vp, _i, _vp, _sz, _vp]),
+    "h3_forward_workspace_size": (_sz, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_io_dims),
+                                        _vp, _i]),
+    "h3_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_io_dims),
+                        ctypes.POINTER(h3_io_weights), ctypes.POINTER(h3_block_weights), _i,
+                        ctypes.POINTER(h3_block_weights), _i, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+                        _vp, _vp, _sz, _vp]),
     "h3_stack_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _i, _vp,
                               _vp, _vp, _i, _vp, _sz, _vp]),
 }
@@ -302,3 +319,34 @@ def h3_stack_forward(dims: h3_dims, weights: Sequence[h3_block_weights], layout:
     _check(lib().h3_stack_forward(ctypes.byref(dims), arr, len(weights), layout.handle,
                                   _ptr(tmod), _ptr(x), B, _ptr(ws), ws_bytes, _stream(stream)),
            "h3_stack_forward")
+
+
+def make_io_dims(d) -> h3_io_dims:
+    """h3_io_dims from any object with video_channels, audio_in_channels,
+    text_dim and final_norm_eps attributes."""
+    return h3_io_dims(video_channels=d.video_channels, audio_channels=d.audio_in_channels,
+                      text_dim=d.text_dim, final_norm_eps=d.final_norm_eps)
+
+
+def make_io_weights(w_patch_video, w_patch_audio, w_text, w_t1, w_t2, w_proj, w_out, out_table,
+                    w_head_video, w_head_audio) -> h3_io_weights:
+    return h3_io_weights(*[_ptr(t) for t in (w_patch_video, w_patch_audio, w_text, w_t1, w_t2,
+                                             w_proj, w_out, out_table, w_head_video,
+                                             w_head_audio)])
+
+
+def h3_forward_workspace_size(dims: h3_dims, io: h3_io_dims, layout: Layout, B: int) -> int:
+    return lib().h3_forward_workspace_size(ctypes.byref(dims), ctypes.byref(io), layout.handle, B)
+
+
+def h3_forward(dims: h3_dims, io: h3_io_dims, io_weights: h3_io_weights,
+               refiner: Sequence[h3_block_weights], blocks: Sequence[h3_block_weights],
+               layout: Layout, timestep, B: int, video, audio, text, video_out, audio_out, ws,
+               ws_bytes: int, stream=None) -> None:
+    ref = (h3_block_weights * max(1, len(refiner)))(*refiner)
+    blk = (h3_block_weights * max(1, len(blocks)))(*blocks)
+    _check(lib().h3_forward(ctypes.byref(dims), ctypes.byref(io), ctypes.byref(io_weights), ref,
+                            len(refiner), blk, len(blocks), layout.handle, _ptr(timestep), B,
+                            _ptr(video), _ptr(audio), _ptr(text), _ptr(video_out),
+                            _ptr(audio_out), _ptr(ws), ws_bytes, _stream(stream)),
+           "h3_forward")

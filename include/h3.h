@@ -281,6 +281,75 @@ H3_API h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* w
                            h3_layout_t layout, const float* tmod, void* x, int B, void* ws,
                            size_t ws_bytes, h3_stream_t stream);
 
+/* ---- the whole transformer forward: the denoiser around the stack ---- */
+
+/* Widths of the rows that enter and leave the transformer (constructor
+ * parameters in_channels * prod(patch_size), audio_in_channels, text_dim and
+ * final_norm_eps). video_channels and audio_channels are 32, 64, 96 or 128;
+ * text_dim % 64 == 0. */
+typedef struct {
+  int video_channels, audio_channels, text_dim;
+  float final_norm_eps;
+} h3_io_dims;
+
+/* Parameters outside the block stack (DEVICE pointers, [out, in] row-major):
+ *   w_patch_video [H, video_channels] f32, w_patch_audio [H, audio_channels] f32:
+ *             the input patch projections (float32 modules, no bias)
+ *   w_text    [H, text_dim] bf16: the text projection (part of the bf16 stack)
+ *   w_t1, w_t2, w_proj: the timestep MLP and the stack's shared AdaLN
+ *             projection, as for h3_timestep_modulation
+ *   w_out     [2H, time_embed_dim] f32: norm_out's (shift, scale) projection of
+ *             SiLU(temb)
+ *   out_table [2, 2, H] f32: norm_out's per-modality rows, (video, audio) x
+ *             (shift, scale)
+ *   w_head_video [video_channels, H] f32, w_head_audio [audio_channels, H] f32:
+ *             the two output heads (float32 modules, no bias) */
+typedef struct {
+  const float* w_patch_video;
+  const float* w_patch_audio;
+  const void* w_text;
+  const float* w_t1;
+  const float* w_t2;
+  const float* w_proj;
+  const float* w_out;
+  const float* out_table;
+  const float* w_head_video;
+  const float* w_head_audio;
+} h3_io_weights;
+
+/* Bytes of device workspace h3_forward needs for B batch elements of the
+ * layout (0 on invalid arguments). */
+H3_API size_t h3_forward_workspace_size(const h3_dims* dims, const h3_io_dims* io,
+                                        h3_layout_t layout, int B);
+
+/* One transformer forward ("MiniMaxH3Transformer3DModel" page, `forward`):
+ * latent rows in, velocities out, each in the row order of its index tensor.
+ *   video [B, n_video, video_channels] f32, audio [B, n_audio, audio_channels]
+ *   f32, text [B, n_text, text_dim] bf16 (the text encoder's condition);
+ *   timestep [n_t] f32 (the distinct values, unscaled in [0, 1]);
+ *   video_out [B, n_video, video_channels] f32, audio_out [B, n_audio,
+ *   audio_channels] f32.
+ * Steps: the timestep MLP, tmod = W_proj SiLU(temb) and norm_out's modulation
+ * W_out SiLU(temb) (fp32); the patch projections (fp32) written into the
+ * stack's fp32 residual stream of valid rows; the text projection, then
+ * n_refiner refiner blocks (the block of this library with its own weights,
+ * over the text rows alone as their own sequence, modulated by the text table
+ * row and the rows' timesteps) and a LayerNorm (no affine, final_norm_eps) into
+ * the stream; n_blocks stack blocks (as h3_stack_forward, the stream staying
+ * fp32); norm_out = LayerNorm (no affine, final_norm_eps) * (1 + scale) + shift
+ * with (shift, scale) = out_table[modality] + W_out SiLU(temb) of the row's
+ * timestep; the fp32 heads. Readings where the page leaves the structure open:
+ * no biases; the refiner's block structure, modulation and output norm and
+ * norm_out's modulation source as just described. Padding rows take no part.
+ * ws: h3_forward_workspace_size bytes. Enqueues only; outputs are written at
+ * stream completion. */
+H3_API h3_status h3_forward(const h3_dims* dims, const h3_io_dims* io, const h3_io_weights* io_weights,
+                            const h3_block_weights* refiner, int n_refiner,
+                            const h3_block_weights* blocks, int n_blocks, h3_layout_t layout,
+                            const float* timestep, int B, const float* video, const float* audio,
+                            const void* text, float* video_out, float* audio_out, void* ws,
+                            size_t ws_bytes, h3_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -354,6 +354,110 @@ def stack_forward(x: np.ndarray, weights_for_block: Callable[[int], object], n_b
 
 
 # --------------------------------------------------------------------------
+# The denoiser around the stack: input projections, text refiner, norm_out and
+# the two output heads  [MX: constructor parameters in_channels,
+# audio_in_channels, patch_size, text_dim, num_refiner_layers, final_norm_eps;
+# the mixed-precision note (patch projections, timestep MLP and output heads
+# in float32); `forward` returns the video and audio velocities in the row
+# order of video_indices and audio_indices]  [ME: "Exacte DiT fusions": final
+# audio / video AdaLN; "Sampler en DiT controls": timestep-aware output head]
+#
+# Readings where the pages leave the structure open: no biases; the text
+# projection belongs to the bf16 stack (it is not among the float32 modules);
+# each refiner block is a block of the stack's structure with its own weights,
+# run over the text rows alone as their own sequence and modulated like the
+# stack (table row of the text tag + the row's timestep); the refiner output is
+# a LayerNorm without affine (eps = final_norm_eps); norm_out is the same
+# LayerNorm followed by a per-modality AdaLN (shift, scale) whose rows are
+# out_table[modality] + W_out . SiLU(temb); the heads are float32 linears.
+# --------------------------------------------------------------------------
+
+def timestep_embedding(t: np.ndarray, w_t1: np.ndarray, w_t2: np.ndarray,
+                       freq_dim: int) -> np.ndarray:
+    """temb[n_t, E] = W_t2 . SiLU(W_t1 . sinusoid(t)): the timestep MLP."""
+    s = timestep_sinusoid(t, freq_dim)
+    return silu(s @ np.asarray(w_t1, F).T) @ np.asarray(w_t2, F).T
+
+
+def output_modulation(t: np.ndarray, w_t1: np.ndarray, w_t2: np.ndarray, w_out: np.ndarray,
+                      freq_dim: int, hidden: int) -> np.ndarray:
+    """tmod_out[n_t, 2, H] = W_out . SiLU(temb): the (shift, scale) of norm_out."""
+    temb = timestep_embedding(t, w_t1, w_t2, freq_dim)
+    return (silu(temb) @ np.asarray(w_out, F).T).reshape(len(t), 2, hidden)
+
+
+def patch_project(latents: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """[n, C] latent rows -> [n, H] = rows . W^T (float32 module, no bias)."""
+    return np.asarray(latents, F) @ np.asarray(w, F).T
+
+
+def text_project(enc_bits: np.ndarray, w_text_bits: np.ndarray) -> np.ndarray:
+    """[n, text_dim] bf16 text condition -> [n, H] with the bf16 [H, text_dim] weight."""
+    return bf16_to_f64(enc_bits) @ bf16_to_f64(w_text_bits).T
+
+
+def text_only_layout(layout):
+    """The text rows of a packed layout as a sequence of their own (index
+    order of text_idx): their positions and timestep indices, tag 1."""
+    from types import SimpleNamespace
+    ti = np.asarray(layout.text_idx)
+    n = ti.shape[0]
+    return SimpleNamespace(tags=np.full(n, 1, np.int32), pos=np.asarray(layout.pos)[ti],
+                           t_idx=np.asarray(layout.t_idx)[ti], timestep=layout.timestep,
+                           text_idx=np.arange(n), video_idx=np.zeros(0, np.int32),
+                           audio_idx=np.zeros(0, np.int32), S=n)
+
+
+def refine_text(xt: np.ndarray, refiner: Sequence, layout, tmod: np.ndarray, dims,
+                final_eps: float) -> np.ndarray:
+    """The refiner blocks over the projected text rows ([n_text, H], text_idx
+    order) as their own sequence, then LayerNorm (no affine, final_norm_eps)."""
+    lt = text_only_layout(layout)
+    y = np.asarray(xt, F)[None]
+    for w in refiner:
+        y = block_forward(y, w, lt, tmod, dims)
+    return layer_norm(y[0], final_eps)
+
+
+def output_head(x_rows: np.ndarray, shift: np.ndarray, scale: np.ndarray, w_head: np.ndarray,
+                final_eps: float) -> np.ndarray:
+    """norm_out then the float32 head: (LN(x) (1 + scale) + shift) . W_head^T."""
+    return norm_modulate(np.asarray(x_rows, F), shift, scale, final_eps) @ np.asarray(w_head, F).T
+
+
+def denoiser_forward(video: np.ndarray, audio: np.ndarray, text: np.ndarray, dw,
+                     blocks: Callable[[int], object], n_blocks: int, layout, dims,
+                     final_eps: float) -> Tuple[np.ndarray, np.ndarray]:
+    """One transformer forward for one batch element: video [n_video, C_v] and
+    audio [n_audio, C_a] latent rows, text [n_text, text_dim] bf16 bits, each in
+    the order of its index tensor -> (video velocity [n_video, C_v], audio
+    velocity [n_audio, C_a]) in the same orders.
+
+    ``dw`` holds w_patch_video, w_patch_audio, w_text, refiner (block weights),
+    w_t1, w_t2, w_proj, w_out, out_table ([2, 2, H]: video, audio x shift,
+    scale), w_head_video, w_head_audio.
+    """
+    H = dims.hidden
+    t = layout.timestep
+    tmod = timestep_modulation(t, dw.w_t1, dw.w_t2, dw.w_proj, dims.freq_dim, H)
+    tmo = output_modulation(t, dw.w_t1, dw.w_t2, dw.w_out, dims.freq_dim, H)
+    x = np.zeros((layout.S, H), F)
+    vi, ai, ti = (np.asarray(a) for a in (layout.video_idx, layout.audio_idx, layout.text_idx))
+    x[vi] = patch_project(video, dw.w_patch_video)
+    x[ai] = patch_project(audio, dw.w_patch_audio)
+    if ti.shape[0]:
+        x[ti] = refine_text(text_project(text, dw.w_text), dw.refiner, layout, tmod, dims,
+                            final_eps)
+    x = stack_forward(x[None], blocks, n_blocks, layout, tmod, dims)[0]
+    t_idx = np.asarray(layout.t_idx)
+    out = []
+    for idx, m, w_head in ((vi, 0, dw.w_head_video), (ai, 1, dw.w_head_audio)):
+        mod = np.asarray(dw.out_table, F)[m][None] + tmo[t_idx[idx]]  # [n, 2, H]
+        out.append(output_head(x[idx], mod[:, 0], mod[:, 1], w_head, final_eps))
+    return out[0], out[1]
+
+
+# --------------------------------------------------------------------------
 # a0 / a1: layout validation, tile classes, compaction, pack / unpack
 #          [MX: forward arguments; caller builds the packing]
 # --------------------------------------------------------------------------

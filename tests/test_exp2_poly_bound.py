@@ -5,7 +5,9 @@ The kernel evaluates part of the softmax exponentials 2^x (x <= 0, clamped at
 1.5 * 2^23, 2^f by a cubic in f on [-1/2, 1/2] (Horner with fused
 multiply-adds), and j added to the exponent field of the result. Its source
 states a maximum relative error of 7.7e-5 wherever 2^x is a normal float32
-(x >= -125; bf16, which stores P, keeps 3.9e-3). This test reads the cubic's coefficients from the kernel source,
+(x >= -125; bf16, which stores P, keeps 3.9e-3). This test reads the cubic's coefficients from the kernel source (the packed
+form computes two values with the same fused multiply-adds, so each lane's
+arithmetic is what is evaluated here),
 evaluates the same float32 steps on the host over a dense grid of
 [-126, 0] and over every float32 f in a fine grid of [-1/2, 1/2], and checks the
 stated bound against numpy's float64 exp2.
@@ -22,14 +24,15 @@ STATED_MAX_REL = 7.7e-5
 
 
 def _coefficients():
+    """The cubic's coefficients kExpC3 .. kExpC0 as the kernel source states them."""
     src = open(SRC).read()
-    body = src[src.index("exp2_poly(float x)"):]
-    body = body[:body.index("\n}")]
-    lits = [float(v) for v in re.findall(r"(-?\d+\.\d+)f", body)]
-    # the clamp (-126), the magic constant, then the cubic's four coefficients
-    coeffs = [v for v in lits if abs(v) < 2.0]
-    assert len(coeffs) == 4, coeffs
-    return coeffs  # c3, c2, c1, c0 in Horner order
+    vals = {}
+    for name in ("kExpC3", "kExpC2", "kExpC1", "kExpC0"):
+        m = re.search(name + r"\s*=\s*(-?\d+\.\d+)f", src)
+        assert m, name
+        vals[name] = float(m.group(1))
+    assert re.search(r"kRoundMagic\s*=\s*12582912\.f", src)
+    return vals["kExpC3"], vals["kExpC2"], vals["kExpC1"], vals["kExpC0"]
 
 
 def _fma32(a, b, c):

@@ -4,6 +4,8 @@ The stack gathers the valid rows once into an fp32 residual stream, runs every
 block on it with no mask, and scatters the result back (rounded to bf16 once).
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -17,6 +19,9 @@ from workloads import (FULL_DIMS, TINY_DIMS, Dims, Layout, activations, block_we
                        config_layout, normal_bf16, prologue_weights, random_layout)
 
 pytestmark = pytest.mark.gpu
+
+GOLDEN5 = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                       "stack_config5_golden.npz")
 
 
 def gpu_stack(dl, dws, tmod, x, B):
@@ -108,31 +113,72 @@ def _valid_only_layout(L):
                   text_idx=np.nonzero(tags == 1)[0].astype(np.int32))
 
 
-def test_stack_config5_50_blocks_properties():
+@pytest.fixture(scope="module")
+def config5():
+    """The config-5 stack on the device: layout, 50 blocks' weights (generated
+    one block at a time and hashed as they go), tmod and the input rows."""
+    from tests.golden.make_stack_config5_golden import InputDigest, layout_digest
+    dims = FULL_DIMS
+    L = config_layout(5)
+    pw = prologue_weights(dims, 5)
+    xb = activations(dims, 5, L.S)
+    dig = InputDigest()
+    layout_digest(dig, L)
+    dig.add(xb)
+    dig.add(pw.w_t1, pw.w_t2, pw.w_proj)
+    dws = []
+    for i in range(50):
+        w = block_weights(dims, 5, i)
+        dig.add_block(w)
+        dws.append(DevWeights(w))
+    return dict(dims=dims, L=L, dl=DevLayout(dims, L), dws=dws, xb=xb,
+                tmod=gpu_tmod(dims, L.timestep, pw), digest=dig.hexdigest())
+
+
+def test_stack_config5_50_blocks_against_float64_golden(config5):
+    """The full-width 50-block stack over the 16384-row padded layout against
+    the float64 oracle's 50-block forward, stored at sampled rows by
+    tests/golden/make_stack_config5_golden.py (rows next to every padding run,
+    in the mixed tiles, at tile edges, and random rows of each modality):
+    x_out and the stack's update x_out - x_in within rel-L2 1e-2 and max-abs
+    5e-2, padding rows bit-identical."""
+    g = np.load(GOLDEN5)
+    assert str(g["input_sha256"]) == config5["digest"], "inputs differ from the golden's"
+    assert int(g["n_blocks"]) == 50
+    L, xb = config5["L"], config5["xb"]
+    rows = g["rows"]
+    np.testing.assert_array_equal(g["x_in_bits"], xb[0, rows])
+    x = dev_bf16(xb)
+    gpu_stack(config5["dl"], config5["dws"], config5["tmod"], x, 1)
+    got = host_f64(x[0, torch.from_numpy(rows).cuda()])
+    ref = g["x_out"].astype(np.float64)
+    x0 = O.bf16_to_f64(xb[0, rows])
+    pad = (L.tags < 0)[rows]
+    assert pad.sum() >= 7 and (~pad).sum() >= 50
+    assert_close(got, ref, what="cfg5 50-block x_out")
+    assert_close(got[~pad] - x0[~pad], ref[~pad] - x0[~pad], what="cfg5 50-block update",
+                 mabs=np.inf)
+    np.testing.assert_array_equal(got[pad], x0[pad])
+    # the stack moved the valid rows far beyond bf16 resolution
+    assert np.linalg.norm(ref[~pad] - x0[~pad]) > 0.5 * np.linalg.norm(x0[~pad])
+
+
+def test_stack_config5_50_blocks_properties(config5):
     """The full 50-block, 16384-row stack: padding rows untouched bit for bit,
     finite outputs, deterministic, and identical (bit for bit) to the same stack
     run on the valid rows alone as a padding-free sequence."""
-    dims = FULL_DIMS
-    L = config_layout(5)
-    dl = DevLayout(dims, L)
-    pw = prologue_weights(dims, 5)
-    dws = [DevWeights(block_weights(dims, 5, i)) for i in range(50)]
-    tmod = gpu_tmod(dims, L.timestep, pw)
-    xb = activations(dims, 5, L.S)
+    dims, L, dws, tmod, xb = (config5[k] for k in ("dims", "L", "dws", "tmod", "xb"))
     x1 = dev_bf16(xb)
-    gpu_stack(dl, dws, tmod, x1, 1)
+    gpu_stack(config5["dl"], dws, tmod, x1, 1)
     out1 = host_bits(x1)[0]
     pad = L.tags < 0
     np.testing.assert_array_equal(out1[pad], xb[0, pad])
     assert np.all(np.isfinite(O.bf16_to_f64(out1)))
     x2 = dev_bf16(xb)
-    gpu_stack(dl, dws, tmod, x2, 1)
+    gpu_stack(config5["dl"], dws, tmod, x2, 1)
     np.testing.assert_array_equal(host_bits(x2)[0], out1)
     Lv = _valid_only_layout(L)
     dlv = DevLayout(dims, Lv)
     xv = dev_bf16(np.ascontiguousarray(xb[:, ~pad]))
     gpu_stack(dlv, dws, tmod, xv, 1)
     np.testing.assert_array_equal(host_bits(xv)[0], out1[~pad])
-    # the stack moved the valid rows well beyond bf16 resolution
-    d = O.bf16_to_f64(out1[~pad]) - O.bf16_to_f64(xb[0, ~pad])
-    assert np.linalg.norm(d) > 0.5 * np.linalg.norm(O.bf16_to_f64(xb[0, ~pad]))

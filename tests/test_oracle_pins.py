@@ -708,3 +708,175 @@ def test_emulated_residual_rounds_after_the_add():
         assert got[0, 0] == want
     got = O.out_project_residual(x, np.array([[1.0]]), np.ones((1, 1)), w_o, emulate=False)
     assert got[0, 0] == 1.001953125
+
+
+# ---------------------------------------------------------------- the denoiser around the stack
+
+def test_golden_denoiser_defaults_match_full_dims():
+    g = _golden()
+    d = FULL_DIMS
+    assert d.in_channels == g["in_channels"] and d.audio_in_channels == g["audio_in_channels"]
+    assert d.patch_size == (g["patch_size_t"], g["patch_size_h"], g["patch_size_w"])
+    assert d.video_channels == g["video_row_channels"] == 96
+    assert d.text_dim == g["text_dim"]
+    assert d.num_refiner_layers == g["num_refiner_layers"]
+    assert d.final_norm_eps == g["final_norm_eps"]
+
+
+def test_timestep_embedding_worked_by_hand():
+    """The same tiny prologue as test_timestep_modulation_worked_by_hand: the
+    MLP output temb at t = 0 is [SiLU(1) - SiLU(0), -2 SiLU(1)]
+    = [0.7310585786, -1.4621171573]; at t = 0.5, [-0.5637917047, -1.2397100173].
+    The output modulation W_out . SiLU(temb) then follows from the SiLU values
+    listed there."""
+    w_t1 = np.array([[1, 0, 0, 0], [0, 0, 2, 100]], F)
+    w_t2 = np.array([[1, -1], [-2, 0]], F)
+    temb = O.timestep_embedding(np.array([0.0, 0.5]), w_t1, w_t2, 4)
+    np.testing.assert_allclose(temb, [[0.7310585786, -1.4621171573],
+                                      [-0.5637917047, -1.2397100173]], atol=1e-9)
+    w_out = np.array([[1, 0], [0, 1], [1, 1], [2, -1]], F)  # 2 chunks of H = 2
+    got = O.output_modulation(np.array([0.0, 0.5]), w_t1, w_t2, w_out, 4, 2)
+    b0 = np.array([0.49349197528601374, -0.2750881684806041])
+    b1 = np.array([-0.20447066856192508, -0.278298119967226])
+    np.testing.assert_allclose(got, np.stack([(w_out @ b).reshape(2, 2) for b in (b0, b1)]),
+                               rtol=1e-9)
+
+
+def test_input_projections_match_torch_linear_and_a_hand_case():
+    g = np.random.default_rng(41)
+    lat = g.standard_normal((7, 96)).astype(np.float32)
+    w = g.standard_normal((64, 96)).astype(np.float32)
+    np.testing.assert_allclose(O.patch_project(lat, w), torch.nn.functional.linear(
+        torch.tensor(lat, dtype=torch.float64), torch.tensor(w, dtype=torch.float64)).numpy(),
+        rtol=1e-12, atol=1e-12)
+    # by hand: rows [1, 2] and [0, -1] through [[1, 0], [1, 1], [0, 3]]
+    np.testing.assert_array_equal(O.patch_project(np.array([[1.0, 2.0], [0.0, -1.0]]),
+                                                  np.array([[1, 0], [1, 1], [0, 3]])),
+                                  [[1, 3, 6], [0, -1, -3]])
+    enc = f32_to_bf16_bits(np.array([[1.0, -2.0, 0.5]], np.float32))
+    wt = f32_to_bf16_bits(np.array([[1, 1, 1], [2, 0, -4]], np.float32))
+    np.testing.assert_array_equal(O.text_project(enc, wt), [[-0.5, 0.0]])
+
+
+def _denoiser_case(seed=0, S=90):
+    d = SMALL
+    d = Dims(**dict(d.__dict__, text_dim=64, num_refiner_layers=2, in_channels=4,
+                    audio_in_channels=8))
+    L = random_layout(S, seed, pad_runs=2, max_run=9, n_t=4)
+    g = np.random.default_rng([seed, 77])
+    from types import SimpleNamespace
+    H, E = d.hidden, d.time_embed_dim
+    dw = SimpleNamespace(
+        w_patch_video=g.standard_normal((H, d.video_channels)) * 0.2,
+        w_patch_audio=g.standard_normal((H, d.audio_in_channels)) * 0.2,
+        w_text=f32_to_bf16_bits((g.standard_normal((H, d.text_dim)) * 0.1).astype(np.float32)),
+        refiner=[_weights_big_gates(d, 200 + i) for i in range(2)],
+        w_t1=g.standard_normal((d.time_hidden, d.freq_dim)) * 0.05,
+        w_t2=g.standard_normal((E, d.time_hidden)) * 0.05,
+        w_proj=g.standard_normal((6 * H, E)) * 0.05,
+        w_out=g.standard_normal((2 * H, E)) * 0.05,
+        out_table=g.standard_normal((2, 2, H)) * 0.2,
+        w_head_video=g.standard_normal((d.video_channels, H)) * 0.1,
+        w_head_audio=g.standard_normal((d.audio_in_channels, H)) * 0.1)
+    blocks = [_weights_big_gates(d, 300 + i) for i in range(2)]
+    video = g.standard_normal((len(L.video_idx), d.video_channels))
+    audio = g.standard_normal((len(L.audio_idx), d.audio_in_channels))
+    text = f32_to_bf16_bits(g.standard_normal((len(L.text_idx), d.text_dim)).astype(np.float32))
+    return d, L, dw, blocks, video, audio, text
+
+
+def test_output_head_is_layer_norm_modulate_then_linear():
+    g = np.random.default_rng(9)
+    x = g.standard_normal((5, 32)) * 3 + 1
+    sh, sc = g.standard_normal((5, 32)), g.standard_normal((5, 32))
+    w = g.standard_normal((6, 32))
+    xt = torch.tensor(x)
+    ln = torch.nn.functional.layer_norm(xt, (32,), eps=1e-5)
+    ref = torch.nn.functional.linear(ln * (1 + torch.tensor(sc)) + torch.tensor(sh),
+                                     torch.tensor(w)).numpy()
+    np.testing.assert_allclose(O.output_head(x, sh, sc, w, 1e-5), ref, rtol=1e-10, atol=1e-12)
+    # a constant row normalises to 0, so the head sees only the shift
+    c = np.full((1, 32), 2.5)
+    np.testing.assert_allclose(O.output_head(c, sh[:1], sc[:1], w, 1e-5), sh[:1] @ w.T,
+                               atol=1e-9)
+
+
+def test_refiner_attends_text_rows_only_and_ends_in_a_layer_norm():
+    d, L, dw, blocks, video, audio, text = _denoiser_case(1)
+    H = d.hidden
+    tmod = O.timestep_modulation(L.timestep, dw.w_t1, dw.w_t2, dw.w_proj, d.freq_dim, H)
+    xt = O.text_project(text, dw.w_text)
+    got = O.refine_text(xt, dw.refiner, L, tmod, d, 1e-5)
+    # the refiner's blocks equal the block run on the text rows as a sequence of their own
+    ti = L.text_idx
+    Lt = make_layout([("text", 0, len(ti))], timesteps="given", t_values=L.timestep,
+                     t_idx=L.t_idx[ti])
+    Lt.pos = L.pos[ti]
+    y = xt[None]
+    for w in dw.refiner:
+        y = O.block_forward(y, w, Lt, tmod, d)
+    np.testing.assert_allclose(got, torch.nn.functional.layer_norm(
+        torch.tensor(y[0]), (H,), eps=1e-5).numpy(), rtol=1e-10, atol=1e-12)
+    # zero gates in the refiner blocks: the output is the LayerNorm of the projection
+    z = [dataclasses_replace_gates(w) for w in dw.refiner]
+    tz = tmod.copy()
+    tz[:, [2, 5]] = 0.0
+    np.testing.assert_allclose(O.refine_text(xt, z, L, tz, d, 1e-5), O.layer_norm(xt, 1e-5),
+                               rtol=1e-12, atol=1e-12)
+
+
+def dataclasses_replace_gates(w):
+    import copy
+    w = copy.copy(w)
+    w.ada_table = np.array(w.ada_table, copy=True)
+    w.ada_table[:, [2, 5]] = 0.0
+    return w
+
+
+def test_denoiser_with_identity_blocks_is_head_of_normed_projection():
+    """With every gate zero (refiner and stack blocks, table and tmod), the
+    blocks pass x through, so the velocity of a video row is the head applied
+    to norm_out of its patch projection: rebuilt here from torch CPU ops."""
+    d, L, dw, blocks, video, audio, text = _denoiser_case(2)
+    dw.refiner = [dataclasses_replace_gates(w) for w in dw.refiner]
+    blocks = [dataclasses_replace_gates(w) for w in blocks]
+    dw.w_proj = np.array(dw.w_proj, copy=True)
+    H = d.hidden
+    for c in (2, 5):
+        dw.w_proj[c * H:(c + 1) * H] = 0.0
+    vv, va = O.denoiser_forward(video, audio, text, dw, lambda i: blocks[i], 2, L, d, 1e-5)
+    tmo = torch.tensor(O.output_modulation(L.timestep, dw.w_t1, dw.w_t2, dw.w_out, d.freq_dim,
+                                           H))
+    for lat, idx, m, wp, wh, got in ((video, L.video_idx, 0, dw.w_patch_video, dw.w_head_video, vv),
+                                     (audio, L.audio_idx, 1, dw.w_patch_audio, dw.w_head_audio, va)):
+        x = torch.nn.functional.linear(torch.tensor(lat), torch.tensor(wp))
+        mod = torch.tensor(dw.out_table)[m][None] + tmo[torch.tensor(L.t_idx[idx]).long()]
+        h = torch.nn.functional.layer_norm(x, (H,), eps=1e-5) * (1 + mod[:, 1]) + mod[:, 0]
+        ref = torch.nn.functional.linear(h, torch.tensor(wh)).numpy()
+        np.testing.assert_allclose(got, ref, rtol=1e-9, atol=1e-11)
+
+
+def test_denoiser_rows_permute_with_their_layout_and_padding_is_inert():
+    d, L, dw, blocks, video, audio, text = _denoiser_case(3)
+    run = lambda L_: O.denoiser_forward(video, audio, text, dw, lambda i: blocks[i], 2, L_, d, 1e-5)
+    vv, va = run(L)
+    assert np.linalg.norm(vv) > 0 and np.linalg.norm(va) > 0
+    perm = np.random.default_rng(5).permutation(L.S)
+    inv = np.argsort(perm)
+    Lp = type(L)(tags=L.tags[perm], pos=L.pos[perm], t_idx=L.t_idx[perm], timestep=L.timestep,
+                 video_idx=inv[L.video_idx].astype(np.int32),
+                 audio_idx=inv[L.audio_idx].astype(np.int32),
+                 text_idx=inv[L.text_idx].astype(np.int32))
+    vp, ap = run(Lp)
+    np.testing.assert_allclose(vp, vv, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(ap, va, rtol=1e-9, atol=1e-11)
+    # padding rows: new positions and timestep indices change nothing
+    Lq = type(L)(tags=L.tags, pos=L.pos.copy(), t_idx=L.t_idx.copy(), timestep=L.timestep,
+                 video_idx=L.video_idx, audio_idx=L.audio_idx, text_idx=L.text_idx)
+    pad = L.tags < 0
+    assert pad.any()
+    Lq.pos[pad] = 17.0
+    Lq.t_idx[pad] = 3
+    vq, aq = run(Lq)
+    np.testing.assert_array_equal(vq, vv)
+    np.testing.assert_array_equal(aq, va)

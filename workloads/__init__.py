@@ -28,4 +28,7 @@ from .h3_workloads import (  # noqa: F401
     prologue_weights,
     activations,
     CONFIG_NAMES,
+    DenoiserWeights,
+    denoiser_weights,
+    denoiser_inputs,
 )

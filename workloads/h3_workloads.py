@@ -52,10 +52,22 @@ class Dims:
     norm_eps: float = 1e-5
     qk_norm_eps: float = 1e-5
     n_modalities: int = 3
+    # the denoiser around the stack
+    in_channels: int = 24
+    patch_size: Tuple[int, int, int] = (1, 2, 2)
+    audio_in_channels: int = 32
+    text_dim: int = 5120
+    num_refiner_layers: int = 2
+    final_norm_eps: float = 1e-5
 
     @property
     def attn_width(self) -> int:
         return self.heads * self.head_dim
+
+    @property
+    def video_channels(self) -> int:
+        """Channels of one patched video latent row: in_channels * prod(patch_size)."""
+        return self.in_channels * int(np.prod(self.patch_size))
 
 
 # Default constructor values of MiniMaxH3Transformer3DModel.
@@ -65,7 +77,7 @@ FULL_DIMS = Dims(hidden=5376, heads=56, head_dim=128, ffn=14336,
 # ffn 1408, time_embed_dim 256; the timestep MLP's hidden width equals the
 # hidden size, as it does at full width.
 TINY_DIMS = Dims(hidden=512, heads=6, head_dim=128, ffn=1408,
-                 time_embed_dim=256, time_hidden=512)
+                 time_embed_dim=256, time_hidden=512, text_dim=384)
 
 
 @dataclasses.dataclass
@@ -330,7 +342,10 @@ def random_layout(S: int, seed: int, pad_runs: int = 2, max_run: int = 40,
 _KEYS: Dict[str, int] = {
     "x": 1, "w_qkv": 10, "q_norm": 11, "k_norm": 12, "w_o": 13, "w13": 14,
     "w2": 15, "ada_table": 16, "w_t1": 20, "w_t2": 21, "w_proj": 22,
+    "video": 30, "audio": 31, "text": 32, "w_patch_video": 40, "w_patch_audio": 41,
+    "w_text": 42, "w_out": 43, "out_table": 44, "w_head_video": 45, "w_head_audio": 46,
 }
+REFINER_BLOCK0 = 1000  # block index of the first refiner block's random streams
 
 WEIGHT_STD = 0.02
 
@@ -368,3 +383,60 @@ def prologue_weights(dims: Dims, cfg: int) -> PrologueWeights:
 def activations(dims: Dims, cfg: int, S: int, B: int = 1, key: int = 0) -> np.ndarray:
     """Packed hidden stream x ~ N(0, 1), bf16 bits, [B, S, H]."""
     return normal_bf16((B, S, dims.hidden), [cfg, _KEYS["x"], key], 1.0)
+
+
+# --------------------------------------------------------------------------
+# The denoiser around the stack
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class DenoiserWeights:
+    """Parameters outside the block stack, [out, in]: float32 patch projections,
+    timestep MLP, output modulation and heads; bf16 text projection; the refiner
+    blocks (BlockWeights)."""
+
+    w_patch_video: np.ndarray  # [H, C_v] f32
+    w_patch_audio: np.ndarray  # [H, C_a] f32
+    w_text: np.ndarray         # [H, text_dim] bf16 bits
+    refiner: List[BlockWeights]
+    w_t1: np.ndarray           # [time_hidden, freq_dim] f32
+    w_t2: np.ndarray           # [time_embed_dim, time_hidden] f32
+    w_proj: np.ndarray         # [6H, time_embed_dim] f32
+    w_out: np.ndarray          # [2H, time_embed_dim] f32: norm_out's (shift, scale)
+    out_table: np.ndarray      # [2, 2, H] f32: (video, audio) x (shift, scale)
+    w_head_video: np.ndarray   # [C_v, H] f32
+    w_head_audio: np.ndarray   # [C_a, H] f32
+
+
+def denoiser_weights(dims: Dims, cfg: int) -> DenoiserWeights:
+    """Random-init parameters outside the stack: matrices ~N(0, 0.02^2) (float32,
+    or bf16 for the text projection), the output AdaLN table ~N(0, 0.02^2)."""
+    H, E = dims.hidden, dims.time_embed_dim
+
+    def s(name: str) -> List[int]:
+        return [cfg, _KEYS[name], 0]
+
+    pw = prologue_weights(dims, cfg)
+    return DenoiserWeights(
+        w_patch_video=normal_f32((H, dims.video_channels), s("w_patch_video"), WEIGHT_STD),
+        w_patch_audio=normal_f32((H, dims.audio_in_channels), s("w_patch_audio"), WEIGHT_STD),
+        w_text=normal_bf16((H, dims.text_dim), s("w_text"), WEIGHT_STD),
+        refiner=[block_weights(dims, cfg, REFINER_BLOCK0 + i)
+                 for i in range(dims.num_refiner_layers)],
+        w_t1=pw.w_t1, w_t2=pw.w_t2, w_proj=pw.w_proj,
+        w_out=normal_f32((2 * H, E), s("w_out"), WEIGHT_STD),
+        out_table=normal_f32((2, 2, H), s("out_table"), WEIGHT_STD),
+        w_head_video=normal_f32((dims.video_channels, H), s("w_head_video"), WEIGHT_STD),
+        w_head_audio=normal_f32((dims.audio_in_channels, H), s("w_head_audio"), WEIGHT_STD),
+    )
+
+
+def denoiser_inputs(dims: Dims, cfg: int, layout: Layout, B: int = 1):
+    """Latent rows of one forward, each in the order of its index tensor:
+    video [B, n_video, C_v] and audio [B, n_audio, C_a] float32 ~N(0, 1), text
+    condition [B, n_text, text_dim] bf16 ~N(0, 1)."""
+    nv, na, nt = (int(np.asarray(a).shape[0]) for a in
+                  (layout.video_idx, layout.audio_idx, layout.text_idx))
+    return (normal_f32((B, nv, dims.video_channels), [cfg, _KEYS["video"], 0], 1.0),
+            normal_f32((B, na, dims.audio_in_channels), [cfg, _KEYS["audio"], 0], 1.0),
+            normal_bf16((B, nt, dims.text_dim), [cfg, _KEYS["text"], 0], 1.0))
