@@ -286,6 +286,7 @@ void h3_layout_destroy(h3_layout_t L) {
   if (!L) return;
   cudaDeviceSynchronize();
   cudaFree(L->block);
+  if (L->extra) cudaFree(L->extra);
   delete L;
 }
 
@@ -560,10 +561,13 @@ h3_status h3_forward(const h3_dims* dims, const h3_io_dims* io, const h3_io_weig
                      const h3_block_weights* refiner, int n_refiner,
                      const h3_block_weights* blocks, int n_blocks, h3_layout_t L,
                      const float* timestep, int B, const float* video, const float* audio,
-                     const void* text, float* video_out, float* audio_out, void* ws,
-                     size_t ws_bytes, h3_stream_t stream) {
+                     const void* text, float* video_out, float* audio_out, float* core_residual,
+                     int core_mode, void* ws, size_t ws_bytes, h3_stream_t stream) {
   H3_TRY(check_dims(dims));
   H3_TRY(check_io(dims, io));
+  if (core_mode < H3_CORE_RUN || core_mode > H3_CORE_REUSE) return H3_ERR_ARG;
+  if (core_mode != H3_CORE_RUN && (!core_residual || !aligned16(core_residual)))
+    return core_residual ? H3_ERR_ALIGN : H3_ERR_ARG;
   if (!L || !iw || n_refiner < 0 || n_blocks < 0 || (n_refiner > 0 && !refiner) ||
       (n_blocks > 0 && !blocks) || !ws)
     return H3_ERR_ARG;
@@ -603,7 +607,12 @@ h3_status h3_forward(const h3_dims* dims, const h3_io_dims* io, const h3_io_weig
                                L->video_idx, L->c_of_row, xc, st));
   H3_CUDA(launch_patch_project(B, L->n_audio, H, V, io->audio_channels, audio, iw->w_patch_audio,
                                L->audio_idx, L->c_of_row, xc, st));
-  if (L->n_text > 0) {
+  const size_t stream_n = (size_t)B * V * H;
+  if (core_mode == H3_CORE_REUSE) {
+    // the stored core residual on the fresh projections (text rows carry no output)
+    H3_CUDA(launch_combine(stream_n, core_residual, 1.f, xc, st));
+  }
+  if (core_mode != H3_CORE_REUSE && L->n_text > 0) {
     // text projection (bf16 weights, fp32 out), the refiner blocks on the text
     // rows alone, and the refiner's output norm into the residual stream
     GemmEpiArgs ea;
@@ -615,8 +624,13 @@ h3_status h3_forward(const h3_dims* dims, const h3_io_dims* io, const h3_io_weig
     H3_CUDA(launch_rows_layer_norm(B, L->n_text, H, V, io->final_norm_eps, fw.text, L->text_idx,
                                    L->c_of_row, xc, st));
   }
-  for (int i = 0; i < n_blocks; ++i)
-    H3_TRY(run_block(d, blocks[i], L->compact_view(), fw.tmod, xc, true, B, w, st));
+  if (core_mode == H3_CORE_STORE && stream_n)
+    H3_CUDA(cudaMemcpyAsync(core_residual, xc, stream_n * 4, cudaMemcpyDeviceToDevice, st));
+  if (core_mode != H3_CORE_REUSE)
+    for (int i = 0; i < n_blocks; ++i)
+      H3_TRY(run_block(d, blocks[i], L->compact_view(), fw.tmod, xc, true, B, w, st));
+  // the core residual: the stack's output minus its input
+  if (core_mode == H3_CORE_STORE) H3_CUDA(launch_combine(stream_n, xc, -1.f, core_residual, st));
   // norm_out and the two heads, in the order of the index tensors
   H3_CUDA(launch_out_head(B, L->n_video, H, V, io->video_channels, io->final_norm_eps, xc,
                           L->video_idx, L->c_of_row, L->t_idx, iw->out_table, fw.tmod_out,
@@ -624,6 +638,123 @@ h3_status h3_forward(const h3_dims* dims, const h3_io_dims* io, const h3_io_weig
   H3_CUDA(launch_out_head(B, L->n_audio, H, V, io->audio_channels, io->final_norm_eps, xc,
                           L->audio_idx, L->c_of_row, L->t_idx, iw->out_table + 2 * H,
                           fw.tmod_out, iw->w_head_audio, audio_out, st));
+  return H3_OK;
+}
+
+}  // extern "C"
+
+// ---- token reduction ----
+
+extern "C" {
+
+h3_status h3_layout_reduce(const h3_dims* dims, h3_layout_t full, const int32_t* target,
+                           h3_stream_t stream, h3_layout_t* out) {
+  if (!out) return H3_ERR_ARG;
+  *out = nullptr;
+  H3_TRY(check_dims(dims));
+  if (!full || (full->S > 0 && !target)) return H3_ERR_ARG;
+  if (!aligned16(target)) return H3_ERR_ALIGN;
+  if (full->red_map) return H3_ERR_ARG;  // a reduced layout is not reduced again
+  cudaStream_t st = as_stream(stream);
+  const int S = full->S;
+  const size_t n = (size_t)(S > 0 ? S : 1);
+  uint8_t* tmp = nullptr;
+  // head [S] u8 | r_tags r_tidx r_src_a r_src_b r_video r_text r_audio [S] i32 | r_pos [3S] f32 | n[4]
+  const size_t sz_h = align256(n), sz_i = align256(n * 4), sz_p = align256(n * 12);
+  if (cudaMalloc(&tmp, sz_h + 7 * sz_i + sz_p + 256) != cudaSuccess) return H3_ERR_CUDA;
+  uint8_t* head = tmp;
+  int32_t* r_tags = reinterpret_cast<int32_t*>(tmp + sz_h);
+  int32_t* r_tidx = reinterpret_cast<int32_t*>(tmp + sz_h + sz_i);
+  int32_t* r_src_a = reinterpret_cast<int32_t*>(tmp + sz_h + 2 * sz_i);
+  int32_t* r_src_b = reinterpret_cast<int32_t*>(tmp + sz_h + 3 * sz_i);
+  int32_t* r_video = reinterpret_cast<int32_t*>(tmp + sz_h + 4 * sz_i);
+  int32_t* r_text = reinterpret_cast<int32_t*>(tmp + sz_h + 5 * sz_i);
+  int32_t* r_audio = reinterpret_cast<int32_t*>(tmp + sz_h + 6 * sz_i);
+  float* r_pos = reinterpret_cast<float*>(tmp + sz_h + 7 * sz_i);
+  int32_t* d_n = reinterpret_cast<int32_t*>(tmp + sz_h + 7 * sz_i + sz_p);
+  h3_status rc = H3_OK;
+  h3_layout_t red = nullptr;
+  do {
+    int hn[4] = {0, 0, 0, 0};
+    if (S > 0) {
+      if (launch_pair_heads(full, target, head, st) != cudaSuccess ||
+          launch_reduce_build(full, head, r_tags, r_tidx, r_pos, r_src_a, r_src_b, r_video,
+                              r_text, r_audio, d_n, st) != cudaSuccess ||
+          cudaMemcpyAsync(hn, d_n, 16, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+          cudaStreamSynchronize(st) != cudaSuccess) {
+        rc = H3_ERR_CUDA;
+        break;
+      }
+    }
+    h3_layout_desc desc{hn[0], full->n_t, hn[1], hn[3], hn[2], r_pos, r_tags, r_tidx, r_video,
+                        r_audio, r_text};
+    if ((rc = h3_layout_prepare(dims, &desc, stream, &red)) != H3_OK) break;
+    const size_t map_b = (size_t)(red->n_valid > 0 ? red->n_valid : 1) * sizeof(int2);
+    if (cudaMalloc(&red->extra, map_b) != cudaSuccess) { rc = H3_ERR_CUDA; break; }
+    red->red_map = static_cast<int2*>(red->extra);
+    red->red_parent_S = full->S;
+    red->red_parent_V = full->n_valid;
+    if (launch_reduce_map(red->S, r_tags, r_src_a, r_src_b, red->c_of_row, full->c_of_row,
+                          red->red_map, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+      rc = H3_ERR_CUDA;
+      break;
+    }
+  } while (0);
+  cudaFree(tmp);
+  if (rc != H3_OK) {
+    h3_layout_destroy(red);
+    return rc;
+  }
+  *out = red;
+  return H3_OK;
+}
+
+size_t h3_stack_reduced_workspace_size(const h3_dims* dims, h3_layout_t full,
+                                       h3_layout_t reduced, int B) {
+  if (check_dims(dims) != H3_OK || check_batch(full, B) != H3_OK || !reduced) return 0;
+  return ws_parts(*dims, B, full->S, nullptr, nullptr) +
+         align256((size_t)B * reduced->n_valid * dims->hidden * 4);
+}
+
+h3_status h3_stack_forward_reduced(const h3_dims* dims, const h3_block_weights* weights,
+                                   int n_blocks, h3_layout_t full, h3_layout_t reduced, int r0,
+                                   int r1, const float* tmod, void* x, int B, void* ws,
+                                   size_t ws_bytes, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!full || !reduced || B < 0 || n_blocks < 0 || r0 < 0 || r1 < 0 || !tmod || !x || !ws ||
+      (n_blocks > 0 && !weights))
+    return H3_ERR_ARG;
+  H3_TRY(check_batch(full, B));
+  if (!reduced->red_map || reduced->red_parent_S != full->S ||
+      reduced->red_parent_V != full->n_valid)
+    return H3_ERR_LAYOUT;
+  for (int i = 0; i < n_blocks; ++i) H3_TRY(check_weights(&weights[i]));
+  if (!aligned16(tmod) || !aligned16(x) || !aligned16(ws)) return H3_ERR_ALIGN;
+  if (ws_bytes < h3_stack_reduced_workspace_size(dims, full, reduced, B)) return H3_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  const h3_dims& d = *dims;
+  const int V = full->n_valid, Vr = reduced->n_valid, H = d.hidden;
+  Workspace w, wr;
+  ws_parts(d, B, full->S, &w, ws);
+  ws_parts(d, B, reduced->S, &wr, ws);  // the reduced blocks' scratch, below w.xc
+  float* xc = static_cast<float*>(w.xc);
+  float* xr = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                       ws_parts(d, B, full->S, nullptr, nullptr));
+  const int a = r0 < n_blocks ? r0 : n_blocks;
+  const int e = r1 < n_blocks ? r1 : n_blocks;
+  H3_CUDA(launch_permute_rows_convert(B, V, full->S, H, full->perm, x, xc, true, st));
+  for (int i = 0; i < a; ++i)
+    H3_TRY(run_block(d, weights[i], full->compact_view(), tmod, xc, true, B, w, st));
+  if (a < e) {
+    H3_CUDA(launch_merge(B, Vr, V, H, reduced->red_map, xc, xr, st));
+    for (int i = a; i < e; ++i)
+      H3_TRY(run_block(d, weights[i], reduced->compact_view(), tmod, xr, true, B, wr, st));
+    H3_CUDA(launch_restore(B, Vr, V, H, reduced->red_map, xr, xc, st));
+  }
+  for (int i = (r1 > a ? r1 : a); i < n_blocks; ++i)
+    H3_TRY(run_block(d, weights[i], full->compact_view(), tmod, xc, true, B, w, st));
+  H3_CUDA(launch_permute_rows_convert(B, V, full->S, H, full->perm, xc, x, false, st));
   return H3_OK;
 }
 

@@ -267,7 +267,27 @@ struct HeadLaunch {
   }
 };
 
+// y[i] = a[i] + s * y[i] over n floats (s = -1: the core residual a - y; the
+// stored residual is added with a = y_old, s = 1 as y = x + r).
+__global__ void k_combine(size_t n4, const float4* __restrict__ a, float s, float4* __restrict__ y) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float4 u = a[i], v = y[i];
+    y[i] = make_float4(u.x + s * v.x, u.y + s * v.y, u.z + s * v.z, u.w + s * v.w);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_combine(size_t n, const float* a, float s, float* y, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const size_t n4 = n / 4;
+  size_t grid = (n4 + 255) / 256;
+  if (grid > (size_t)num_sms() * 16) grid = (size_t)num_sms() * 16;
+  k_combine<<<(unsigned)grid, 256, 0, st>>>(n4, reinterpret_cast<const float4*>(a), s,
+                                            reinterpret_cast<float4*>(y));
+  return cudaGetLastError();
+}
 
 bool io_channels_supported(int C) { return C == 32 || C == 64 || C == 96 || C == 128; }
 

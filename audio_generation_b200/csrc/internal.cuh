@@ -60,6 +60,11 @@ struct h3_layout {
   uint8_t* t_tile_class = nullptr;
   uint32_t* t_key_valid = nullptr;
   int t_tiles = 0;
+  // a token-reduced layout (from h3_layout_reduce): for each of its compact
+  // rows, the source rows in its parent's compact stream (second -1 if single)
+  void* extra = nullptr;
+  int2* red_map = nullptr;
+  int red_parent_S = -1, red_parent_V = -1;
   int* err = nullptr;
   std::vector<uint8_t> tile_class_host;
 
@@ -148,7 +153,24 @@ cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, 
 
 int num_sms();
 
+// ---- token reduction (reduce.cu) ----
+cudaError_t launch_pair_heads(const h3_layout* L, const int32_t* target, uint8_t* head,
+                              cudaStream_t st);
+cudaError_t launch_reduce_build(const h3_layout* L, const uint8_t* head, int32_t* r_tags,
+                                int32_t* r_tidx, float* r_pos, int32_t* r_src_a, int32_t* r_src_b,
+                                int32_t* r_video, int32_t* r_text, int32_t* r_audio,
+                                int32_t* out_n, cudaStream_t st);
+cudaError_t launch_reduce_map(int Sr, const int32_t* r_tags, const int32_t* src_a,
+                              const int32_t* src_b, const int32_t* c_of_row_r,
+                              const int32_t* c_of_row_full, int2* map, cudaStream_t st);
+cudaError_t launch_merge(int B, int Vr, int V, int H, const int2* map, const float* xc,
+                         float* xr, cudaStream_t st);
+cudaError_t launch_restore(int B, int Vr, int V, int H, const int2* map, const float* xr,
+                           float* xc, cudaStream_t st);
+
 // ---- the denoiser around the stack (denoiser.cu) ----
+// y = a + s y elementwise over n floats (n % 4 == 0, 16-byte aligned).
+cudaError_t launch_combine(size_t n, const float* a, float s, float* y, cudaStream_t st);
 // Latent / velocity row widths the projection and head kernels take.
 bool io_channels_supported(int C);
 // xc[b, c_of_row[idx[i]]] = W . lat[b, i] (fp32; lat [B, n, C], W [H, C]).

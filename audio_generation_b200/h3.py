@@ -96,12 +96,16 @@ _SIGNATURES = {
                                   _vp]),
     "h3_block_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _vp,
                               _vp, _vp, _i, _vp, _sz, _vp]),
+    "h3_layout_reduce": (_i, [ctypes.POINTER(h3_dims), _vp, _vp, _vp, ctypes.POINTER(_vp)]),
+    "h3_stack_reduced_workspace_size": (_sz, [ctypes.POINTER(h3_dims), _vp, _vp, _i]),
+    "h3_stack_forward_reduced": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights),
+                                      _i, _vp, _vp, _i, _i, _vp, _vp, _i, _vp, _sz, _vp]),
     "h3_forward_workspace_size": (_sz, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_io_dims),
                                         _vp, _i]),
     "h3_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_io_dims),
                         ctypes.POINTER(h3_io_weights), ctypes.POINTER(h3_block_weights), _i,
                         ctypes.POINTER(h3_block_weights), _i, _vp, _vp, _i, _vp, _vp, _vp, _vp,
-                        _vp, _vp, _sz, _vp]),
+                        _vp, _vp, _i, _vp, _sz, _vp]),
     "h3_stack_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _i, _vp,
                               _vp, _vp, _i, _vp, _sz, _vp]),
 }
@@ -339,14 +343,39 @@ def h3_forward_workspace_size(dims: h3_dims, io: h3_io_dims, layout: Layout, B: 
     return lib().h3_forward_workspace_size(ctypes.byref(dims), ctypes.byref(io), layout.handle, B)
 
 
+H3_CORE_RUN, H3_CORE_STORE, H3_CORE_REUSE = 0, 1, 2
+
+
 def h3_forward(dims: h3_dims, io: h3_io_dims, io_weights: h3_io_weights,
                refiner: Sequence[h3_block_weights], blocks: Sequence[h3_block_weights],
                layout: Layout, timestep, B: int, video, audio, text, video_out, audio_out, ws,
-               ws_bytes: int, stream=None) -> None:
+               ws_bytes: int, stream=None, core_residual=None, core_mode: int = 0) -> None:
     ref = (h3_block_weights * max(1, len(refiner)))(*refiner)
     blk = (h3_block_weights * max(1, len(blocks)))(*blocks)
     _check(lib().h3_forward(ctypes.byref(dims), ctypes.byref(io), ctypes.byref(io_weights), ref,
                             len(refiner), blk, len(blocks), layout.handle, _ptr(timestep), B,
                             _ptr(video), _ptr(audio), _ptr(text), _ptr(video_out),
-                            _ptr(audio_out), _ptr(ws), ws_bytes, _stream(stream)),
+                            _ptr(audio_out), _ptr(core_residual), core_mode, _ptr(ws), ws_bytes,
+                            _stream(stream)),
            "h3_forward")
+
+
+def h3_layout_reduce(dims: h3_dims, full: Layout, target, stream=None) -> Layout:
+    out = ctypes.c_void_p()
+    _check(lib().h3_layout_reduce(ctypes.byref(dims), full.handle, _ptr(target),
+                                  _stream(stream), ctypes.byref(out)), "h3_layout_reduce")
+    return Layout(out.value, -1)
+
+
+def h3_stack_reduced_workspace_size(dims: h3_dims, full: Layout, reduced: Layout, B: int) -> int:
+    return lib().h3_stack_reduced_workspace_size(ctypes.byref(dims), full.handle, reduced.handle, B)
+
+
+def h3_stack_forward_reduced(dims: h3_dims, weights: Sequence[h3_block_weights], full: Layout,
+                             reduced: Layout, r0: int, r1: int, tmod, x, B: int, ws, ws_bytes: int,
+                             stream=None) -> None:
+    arr = (h3_block_weights * max(1, len(weights)))(*weights)
+    _check(lib().h3_stack_forward_reduced(ctypes.byref(dims), arr, len(weights), full.handle,
+                                          reduced.handle, r0, r1, _ptr(tmod), _ptr(x), B, _ptr(ws),
+                                          ws_bytes, _stream(stream)),
+           "h3_stack_forward_reduced")

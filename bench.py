@@ -675,6 +675,106 @@ def run_stack(args):
     return 0
 
 
+FORWARD_WORKLOAD = ("full MiniMax-H3 transformer forward: fp32 patch projections (96 / 32 "
+                    "channels), text projection (5120) and 2 refiner blocks, the 50-block stack "
+                    "over the 16384-row padded layout (15872 valid rows, two timesteps), norm_out "
+                    "and the fp32 video / audio heads")
+
+
+def run_forward(args):
+    """--forward: one whole transformer forward (h3_forward) on one GPU, from
+    latent rows to velocities. Prints one JSON line: forward time, valid rows/s
+    and TFLOP/s over the algorithmic flops of the stack, the refiner (over the
+    text rows) and the projections and heads."""
+    import torch
+    from audio_generation_b200 import h3
+    from workloads import denoiser_inputs, denoiser_weights
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    dims = FULL_DIMS
+    d, io = h3.make_dims(dims), h3.make_io_dims(dims)
+    L = config_layout(STACK_CFG)
+    S, V = L.S, L.n_valid
+    nt_rows = len(L.text_idx)
+    bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(
+        torch.bfloat16)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+    def dev_block(w):
+        t = {k: bits(getattr(w, k)) for k in ("w_qkv", "q_norm", "k_norm", "w_o", "w13", "w2")}
+        t["ada_table"] = f32(w.ada_table)
+        return t, h3.make_block_weights(t["w_qkv"], t["q_norm"], t["k_norm"], t["w_o"], t["w13"],
+                                        t["w2"], t["ada_table"])
+
+    keep, blocks = [], []
+    for i in range(STACK_BLOCKS):
+        t, c = dev_block(block_weights(dims, STACK_CFG, i))
+        keep.append(t)
+        blocks.append(c)
+    dw = denoiser_weights(dims, STACK_CFG)
+    refiner = []
+    for w in dw.refiner:
+        t, c = dev_block(w)
+        keep.append(t)
+        refiner.append(c)
+    iot = [f32(dw.w_patch_video), f32(dw.w_patch_audio), bits(dw.w_text), f32(dw.w_t1),
+           f32(dw.w_t2), f32(dw.w_proj), f32(dw.w_out), f32(dw.out_table), f32(dw.w_head_video),
+           f32(dw.w_head_audio)]
+    iw = h3.make_io_weights(*iot)
+    layout = h3.h3_layout_prepare(d, S, L.n_t, f32(L.pos), i32(L.tags), i32(L.t_idx),
+                                  i32(L.video_idx), i32(L.audio_idx), i32(L.text_idx))
+    video, audio, text = denoiser_inputs(dims, STACK_CFG, L)
+    v_d, a_d, t_d, ts = f32(video), f32(audio), bits(text), f32(L.timestep)
+    vo = torch.empty((1, len(L.video_idx), dims.video_channels), device=device)
+    ao = torch.empty((1, len(L.audio_idx), dims.audio_in_channels), device=device)
+    ws_b = h3.h3_forward_workspace_size(d, io, layout, 1)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def forward():
+        h3.h3_forward(d, io, iw, refiner, blocks, layout, ts, 1, v_d, a_d, t_d, vo, ao, ws, ws_b,
+                      stream)
+
+    for _ in range(args.warmup):
+        forward()
+    torch.cuda.synchronize(device)
+    gpu_id = torch.cuda.get_device_properties(device).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        time.sleep(0.3)
+        e0.record(stream)
+        for _ in range(args.steps):
+            forward()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    if h3.h3_layout_error(layout) != h3.H3_OK:
+        raise RuntimeError("device error word set during the forward run")
+    ms = e0.elapsed_time(e1) / args.steps
+    H = dims.hidden
+    flops = (STACK_BLOCKS * block_flops(dims, V) + 2 * block_flops(dims, nt_rows)
+             + 2.0 * nt_rows * dims.text_dim * H
+             + 2.0 * 2 * H * (len(L.video_idx) * dims.video_channels
+                              + len(L.audio_idx) * dims.audio_in_channels))
+    peaks = load_peaks()
+    tflops = flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "valid packed rows/s per transformer forward (bf16 stack, 1xB200)",
+        "value": V / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights and latents)",
+        "config": {"workload": FORWARD_WORKLOAD, "S": S, "valid_rows": V, "blocks": STACK_BLOCKS,
+                   "refiner_blocks": len(refiner), "text_rows": nt_rows, "n_t": int(L.n_t)},
+        "tflops": tflops, "frac_of_sustained_peak": tflops / peaks["bf16_tflops_sustained"],
+        "frac_of_burst_peak": tflops / peaks["bf16_tflops"], "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    layout.close()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -690,6 +790,8 @@ def main(argv=None):
                     help="skip the masked-attention measurement on the padded layout")
     ap.add_argument("--stack", action="store_true",
                     help="time the 50-block stack forward instead (one GPU, own JSON line)")
+    ap.add_argument("--forward", action="store_true",
+                    help="time the whole transformer forward instead (one GPU, own JSON line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -698,6 +800,8 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.stack:
         return run_stack(args)
+    if args.forward:
+        return run_forward(args)
     return run_gpu(args, world, rank, local)
 
 

@@ -281,6 +281,40 @@ H3_API h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* w
                            h3_layout_t layout, const float* tmod, void* x, int B, void* ws,
                            size_t ws_bytes, h3_stream_t stream);
 
+/* ---- token reduction in the middle blocks ---- */
+
+/* Build the token-reduced layout of `full` ("MiniMax H3 Inference Engine voor
+ * Mac computers", section "Token-reduction internals": adjacent horizontal
+ * target-video tokens are paired in the middle blocks; text, audio and
+ * reference tokens stay exact). target [S] i32 (DEVICE): nonzero marks a
+ * target-video row (a row being generated; reference / conditioning frames are
+ * 0). Packed rows r, r + 1 pair when both are target-video rows with the same
+ * t_idx, the same t and h and w coordinates 2k and 2k + 1 (reading: the page
+ * names the pairing, not its rule). The reduced sequence keeps every other row
+ * in packed order; a pair becomes one row at the first row's place with the
+ * mean of the two positions. Returns a layout object usable by every call that
+ * takes a layout, which also records its rows' sources in `full`. Synchronises
+ * `stream`; allocates small device tables, released by h3_layout_destroy. */
+H3_API h3_status h3_layout_reduce(const h3_dims* dims, h3_layout_t full, const int32_t* target,
+                                  h3_stream_t stream, h3_layout_t* out);
+
+/* Workspace bytes of h3_stack_forward_reduced: h3_workspace_size of the full
+ * sequence plus the reduced fp32 stream. */
+H3_API size_t h3_stack_reduced_workspace_size(const h3_dims* dims, h3_layout_t full,
+                                              h3_layout_t reduced, int B);
+
+/* n_blocks blocks as h3_stack_forward, with blocks [r0, r1) run on the reduced
+ * sequence: after block r0 - 1 the fp32 stream is kept as the bypass and each
+ * pair's rows are merged (mean); before block r1 every full row gets its reduced
+ * row's change since the merge added to the bypass (both rows of a pair the same
+ * change). r0 >= r1 runs the plain stack. (The page pairs after block 3 and
+ * restores before block 40, or 30 after the first ten noisy evaluations: r0 =
+ * 3, r1 = 39 or 29 in 0-based block indices.) x [B, S, H] bf16 in place. */
+H3_API h3_status h3_stack_forward_reduced(const h3_dims* dims, const h3_block_weights* weights,
+                                          int n_blocks, h3_layout_t full, h3_layout_t reduced,
+                                          int r0, int r1, const float* tmod, void* x, int B,
+                                          void* ws, size_t ws_bytes, h3_stream_t stream);
+
 /* ---- the whole transformer forward: the denoiser around the stack ---- */
 
 /* Widths of the rows that enter and leave the transformer (constructor
@@ -317,6 +351,16 @@ typedef struct {
   const float* w_head_audio;
 } h3_io_weights;
 
+/* Core residual reuse ("MiniMax H3 Inference Engine voor Mac computers",
+ * section "Sampler en DiT controls": the previous full transformer residual is
+ * held while the patch projections and the timestep-aware head are refreshed).
+ * The core is the text refiner and the block stack; its residual is the stack's
+ * output minus its input, core_residual [B, V, H] f32 over the V valid rows in
+ * packed order. H3_CORE_RUN: a plain forward; H3_CORE_STORE: a plain forward
+ * that also writes core_residual; H3_CORE_REUSE: the refiner and the stack do
+ * not run, the stream is the fresh patch projections plus core_residual. */
+enum { H3_CORE_RUN = 0, H3_CORE_STORE = 1, H3_CORE_REUSE = 2 };
+
 /* Bytes of device workspace h3_forward needs for B batch elements of the
  * layout (0 on invalid arguments). */
 H3_API size_t h3_forward_workspace_size(const h3_dims* dims, const h3_io_dims* io,
@@ -341,14 +385,16 @@ H3_API size_t h3_forward_workspace_size(const h3_dims* dims, const h3_io_dims* i
  * timestep; the fp32 heads. Readings where the page leaves the structure open:
  * no biases; the refiner's block structure, modulation and output norm and
  * norm_out's modulation source as just described. Padding rows take no part.
- * ws: h3_forward_workspace_size bytes. Enqueues only; outputs are written at
- * stream completion. */
+ * core_residual / core_mode: see H3_CORE_RUN (core_residual may be NULL with
+ * H3_CORE_RUN). ws: h3_forward_workspace_size bytes. Enqueues only; outputs
+ * are written at stream completion. */
 H3_API h3_status h3_forward(const h3_dims* dims, const h3_io_dims* io, const h3_io_weights* io_weights,
                             const h3_block_weights* refiner, int n_refiner,
                             const h3_block_weights* blocks, int n_blocks, h3_layout_t layout,
                             const float* timestep, int B, const float* video, const float* audio,
-                            const void* text, float* video_out, float* audio_out, void* ws,
-                            size_t ws_bytes, h3_stream_t stream);
+                            const void* text, float* video_out, float* audio_out,
+                            float* core_residual, int core_mode, void* ws, size_t ws_bytes,
+                            h3_stream_t stream);
 
 #ifdef __cplusplus
 }

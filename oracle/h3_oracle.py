@@ -427,7 +427,8 @@ def output_head(x_rows: np.ndarray, shift: np.ndarray, scale: np.ndarray, w_head
 
 def denoiser_forward(video: np.ndarray, audio: np.ndarray, text: np.ndarray, dw,
                      blocks: Callable[[int], object], n_blocks: int, layout, dims,
-                     final_eps: float) -> Tuple[np.ndarray, np.ndarray]:
+                     final_eps: float, core_residual: Optional[np.ndarray] = None,
+                     reuse: bool = False) -> Tuple[np.ndarray, np.ndarray]:
     """One transformer forward for one batch element: video [n_video, C_v] and
     audio [n_audio, C_a] latent rows, text [n_text, text_dim] bf16 bits, each in
     the order of its index tensor -> (video velocity [n_video, C_v], audio
@@ -436,6 +437,15 @@ def denoiser_forward(video: np.ndarray, audio: np.ndarray, text: np.ndarray, dw,
     ``dw`` holds w_patch_video, w_patch_audio, w_text, refiner (block weights),
     w_t1, w_t2, w_proj, w_out, out_table ([2, 2, H]: video, audio x shift,
     scale), w_head_video, w_head_audio.
+
+    Core residual reuse ([ME] "Sampler en DiT controls": the previous full
+    transformer residual is held while the patch projections and the
+    timestep-aware head are refreshed; reading: the core is the refiner and the
+    block stack, its residual the stack's output minus the stack's input, [S, H];
+    the text rows carry no output, so only video and audio rows use it): with
+    ``core_residual`` given and ``reuse`` False the forward also stores that
+    residual in it; with ``reuse`` True the core does not run and the stream is
+    the fresh projections plus the stored residual.
     """
     H = dims.hidden
     t = layout.timestep
@@ -445,16 +455,119 @@ def denoiser_forward(video: np.ndarray, audio: np.ndarray, text: np.ndarray, dw,
     vi, ai, ti = (np.asarray(a) for a in (layout.video_idx, layout.audio_idx, layout.text_idx))
     x[vi] = patch_project(video, dw.w_patch_video)
     x[ai] = patch_project(audio, dw.w_patch_audio)
-    if ti.shape[0]:
-        x[ti] = refine_text(text_project(text, dw.w_text), dw.refiner, layout, tmod, dims,
-                            final_eps)
-    x = stack_forward(x[None], blocks, n_blocks, layout, tmod, dims)[0]
+    if reuse:
+        x = x + core_residual
+    else:
+        if ti.shape[0]:
+            x[ti] = refine_text(text_project(text, dw.w_text), dw.refiner, layout, tmod, dims,
+                                final_eps)
+        x_in = x.copy()
+        x = stack_forward(x[None], blocks, n_blocks, layout, tmod, dims)[0]
+        if core_residual is not None:
+            core_residual[...] = x - x_in
     t_idx = np.asarray(layout.t_idx)
     out = []
     for idx, m, w_head in ((vi, 0, dw.w_head_video), (ai, 1, dw.w_head_audio)):
         mod = np.asarray(dw.out_table, F)[m][None] + tmo[t_idx[idx]]  # [n, 2, H]
         out.append(output_head(x[idx], mod[:, 0], mod[:, 1], w_head, final_eps))
     return out[0], out[1]
+
+
+# --------------------------------------------------------------------------
+# Token reduction in the middle blocks  [ME: "Token-reduction internals": after
+# block 3 adjacent horizontal target-video tokens are paired, text, audio and
+# reference tokens stay exact; the full-resolution state is kept as a bypass
+# and restored before a later block (40, then 30)]
+#
+# Readings where the page leaves the steps open: a pair is two packed rows r,
+# r + 1 that are both target-video rows with the same t_idx, the same t and h
+# coordinates and w coordinates 2k and 2k + 1; the merged row is the mean of the
+# pair's rows, at the mean of their positions, in the place of the first; at
+# the restore point each row of a pair receives the pair's update (the merged
+# row's change since the merge), added to the bypass; unpaired rows map one to
+# one. Blocks [r0, r1) run on the reduced sequence.
+# --------------------------------------------------------------------------
+
+def reduction_pairs(layout, target: np.ndarray) -> np.ndarray:
+    """Packed rows that head a pair (their partner is the next row)."""
+    tags = np.asarray(layout.tags)
+    pos = np.asarray(layout.pos, F)
+    ti = np.asarray(layout.t_idx)
+    tg = np.asarray(target, bool) & (tags == 0)
+    S = tags.shape[0]
+    heads = []
+    r = 0
+    while r + 1 < S:
+        w = pos[r, 2]
+        if (tg[r] and tg[r + 1] and ti[r] == ti[r + 1] and pos[r, 0] == pos[r + 1, 0]
+                and pos[r, 1] == pos[r + 1, 1] and w % 2 == 0 and pos[r + 1, 2] == w + 1):
+            heads.append(r)
+            r += 2
+        else:
+            r += 1
+    return np.asarray(heads, np.int64)
+
+
+def reduced_layout(layout, heads: np.ndarray):
+    """The sequence with each pair replaced by one row at the first row's place:
+    the pair's tag and timestep index and the mean of the two positions.
+    Returns (layout, rows) with rows[j] = (first packed row, second or -1)."""
+    from types import SimpleNamespace
+    S = len(layout.tags)
+    tail = np.zeros(S, bool)
+    tail[np.asarray(heads, np.int64) + 1] = True
+    is_head = np.zeros(S, bool)
+    is_head[np.asarray(heads, np.int64)] = True
+    keep = np.nonzero(~tail)[0]
+    rows = np.stack([keep, np.where(is_head[keep], keep + 1, -1)], 1)
+    pos = np.asarray(layout.pos, F)[keep].copy()
+    h = is_head[keep]
+    pos[h] = 0.5 * (pos[h] + np.asarray(layout.pos, F)[keep[h] + 1])
+    tags = np.asarray(layout.tags)[keep]
+    return SimpleNamespace(tags=tags, pos=pos, t_idx=np.asarray(layout.t_idx)[keep],
+                           timestep=layout.timestep, S=len(keep),
+                           video_idx=np.nonzero(tags == 0)[0], audio_idx=np.nonzero(tags == 2)[0],
+                           text_idx=np.nonzero(tags == 1)[0]), rows
+
+
+def merge_rows(x: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """x [S, H] -> [len(rows), H]: a pair's rows averaged, other rows copied."""
+    a, b = rows[:, 0], rows[:, 1]
+    out = np.array(x[a], F, copy=True)
+    p = b >= 0
+    out[p] = 0.5 * (x[a[p]] + x[b[p]])
+    return out
+
+
+def restore_rows(bypass: np.ndarray, x_red: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """The full-resolution state: the bypass plus, for every row, the change of
+    its reduced row since the merge (both rows of a pair get the same change)."""
+    d = x_red - merge_rows(bypass, rows)
+    out = np.array(bypass, F, copy=True)
+    out[rows[:, 0]] += d
+    p = rows[:, 1] >= 0
+    out[rows[p, 1]] += d[p]
+    return out
+
+
+def stack_forward_reduced(x: np.ndarray, weights_for_block: Callable[[int], object],
+                          n_blocks: int, layout, tmod: np.ndarray, dims, target: np.ndarray,
+                          r0: int, r1: int) -> np.ndarray:
+    """The stack with blocks [r0, r1) on the token-reduced sequence (B = 1)."""
+    y = np.asarray(x, F)
+    heads = reduction_pairs(layout, target)
+    red, rows = reduced_layout(layout, heads)
+    for i in range(min(r0, n_blocks)):
+        y = block_forward(y, weights_for_block(i), layout, tmod, dims)
+    if r0 < min(r1, n_blocks):
+        bypass = y[0]
+        z = merge_rows(bypass, rows)[None]
+        for i in range(r0, min(r1, n_blocks)):
+            z = block_forward(z, weights_for_block(i), red, tmod, dims)
+        y = restore_rows(bypass, z[0], rows)[None]
+    for i in range(max(r1, r0), n_blocks):
+        y = block_forward(y, weights_for_block(i), layout, tmod, dims)
+    return y
 
 
 # --------------------------------------------------------------------------

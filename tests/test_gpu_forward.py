@@ -137,3 +137,55 @@ def test_forward_full_width_ragged():
     rv, ra = oracle_forward(dims, L, dw, blocks, video, audio, text)
     _check(vo[0], rv, "full-width video velocity")
     _check(ao[0], ra, "full-width audio velocity")
+
+
+def test_forward_core_residual_store_and_reuse():
+    """H3_CORE_STORE gives the plain forward's velocities and the stack's
+    residual (output minus input, valid rows in packed order); H3_CORE_REUSE with
+    fresh latents matches the oracle's reuse of that residual."""
+    dims = Dims(hidden=256, heads=2, head_dim=128, ffn=384, time_embed_dim=64, time_hidden=128,
+                text_dim=128, in_channels=8, audio_in_channels=64)
+    L, dw, blocks = _amplified_case(4, 250, dims)
+    g = np.random.default_rng(90)
+    video = g.standard_normal((1, len(L.video_idx), dims.video_channels)).astype(np.float32)
+    audio = g.standard_normal((1, len(L.audio_idx), dims.audio_in_channels)).astype(np.float32)
+    txt = f32_to_bf16_bits(g.standard_normal((1, len(L.text_idx), dims.text_dim)).astype(np.float32))
+    dl = DevLayout(dims, L)
+    io = h3.make_io_dims(dims)
+    keep = [dev_f32(dw.w_patch_video), dev_f32(dw.w_patch_audio), dev_bf16(dw.w_text),
+            dev_f32(dw.w_t1), dev_f32(dw.w_t2), dev_f32(dw.w_proj), dev_f32(dw.w_out),
+            dev_f32(dw.out_table), dev_f32(dw.w_head_video), dev_f32(dw.w_head_audio)]
+    iw = h3.make_io_weights(*keep)
+    ref = [DevWeights(w) for w in dw.refiner]
+    blk = [DevWeights(w) for w in blocks]
+    V = L.n_valid
+    res = torch.zeros((1, V, dims.hidden), device="cuda")
+    ws_b = h3.h3_forward_workspace_size(dl.dims, io, dl.handle, 1)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+
+    def run(v, a, mode):
+        vo = torch.empty((1, len(L.video_idx), dims.video_channels), device="cuda")
+        ao = torch.empty((1, len(L.audio_idx), dims.audio_in_channels), device="cuda")
+        h3.h3_forward(dl.dims, io, iw, [w.c for w in ref], [w.c for w in blk], dl.handle,
+                      dev_f32(L.timestep), 1, dev_f32(v), dev_f32(a), dev_bf16(txt), vo, ao, ws,
+                      ws_b, core_residual=res, core_mode=mode)
+        torch.cuda.synchronize()
+        assert h3.h3_layout_error(dl.handle) == h3.H3_OK
+        return vo.double().cpu().numpy()[0], ao.double().cpu().numpy()[0]
+
+    v_run, a_run = run(video, audio, h3.H3_CORE_RUN)
+    v_st, a_st = run(video, audio, h3.H3_CORE_STORE)
+    np.testing.assert_array_equal(v_st, v_run)
+    np.testing.assert_array_equal(a_st, a_run)
+    ores = np.zeros((L.S, dims.hidden))
+    O.denoiser_forward(video[0], audio[0], txt[0], dw, lambda i: blocks[i], len(blocks), L, dims,
+                       dims.final_norm_eps, core_residual=ores)
+    valid = np.nonzero(L.tags >= 0)[0]
+    _check(res.double().cpu().numpy()[0], ores[valid], "core residual")
+    v2 = (video * 0.5 + 0.2).astype(np.float32)
+    a2 = (audio * -0.7).astype(np.float32)
+    v_re, a_re = run(v2, a2, h3.H3_CORE_REUSE)
+    rv, ra = O.denoiser_forward(v2[0], a2[0], txt[0], dw, lambda i: blocks[i], len(blocks), L,
+                                dims, dims.final_norm_eps, core_residual=ores, reuse=True)
+    _check(v_re, rv, "reused video velocity")
+    _check(a_re, ra, "reused audio velocity")

@@ -1,0 +1,110 @@
+"""Token reduction in the middle blocks (h3_layout_reduce,
+h3_stack_forward_reduced) against the oracle's stack_forward_reduced.
+
+Source: "MiniMax H3 Inference Engine voor Mac computers", section
+"Token-reduction internals" (adjacent horizontal target-video tokens paired in
+the middle blocks, the full-resolution state kept as a bypass and restored).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from audio_generation_b200 import h3
+from oracle import h3_oracle as O
+from tests.h3_testlib import (DevLayout, DevWeights, assert_close, dev_bf16, dev_f32, dev_i32,
+                              host_bits, host_f64)
+from tests.test_gpu_block import amplified_weights
+from workloads import FULL_DIMS, Dims, block_weights, make_layout, normal_bf16
+
+pytestmark = pytest.mark.gpu
+
+SMALL_W = Dims(hidden=256, heads=2, head_dim=128, ffn=384, time_embed_dim=64, time_hidden=128)
+
+
+def _layout(segs, n_target_from_frame=1):
+    L0 = make_layout(segs, seed=[5])
+    target = (L0.tags == 0) & (L0.pos[:, 0] >= n_target_from_frame)
+    t_idx = (target | (L0.tags == 2)).astype(np.int32)
+    L = make_layout(segs, timesteps="given", t_values=np.array([0.0, 0.6], np.float32),
+                    t_idx=t_idx)
+    return L, target
+
+
+def _run(dims, L, target, ws_host, tmod, xb, r0, r1):
+    dl = DevLayout(dims, L)
+    red = h3.h3_layout_reduce(dl.dims, dl.handle, dev_i32(target.astype(np.int32)))
+    dws = [DevWeights(w) for w in ws_host]
+    x = dev_bf16(xb)
+    ws_b = h3.h3_stack_reduced_workspace_size(dl.dims, dl.handle, red, xb.shape[0])
+    ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+    h3.h3_stack_forward_reduced(dl.dims, [w.c for w in dws], dl.handle, red, r0, r1,
+                                dev_f32(tmod), x, xb.shape[0], ws, ws_b)
+    torch.cuda.synchronize()
+    assert h3.h3_layout_error(dl.handle) == h3.H3_OK
+    return x, dl, red, dws
+
+
+def test_reduced_layout_tables_match_the_oracle():
+    segs = [("text", 0, 70), ("video", (3, 4, 10), 0, 3), ("pad", 40), ("audio", 0, 90),
+            ("pad", 3)]
+    L, target = _layout(segs)
+    dl = DevLayout(SMALL_W, L)
+    red = h3.h3_layout_reduce(dl.dims, dl.handle, dev_i32(target.astype(np.int32)))
+    heads = O.reduction_pairs(L, target)
+    assert heads.size == 2 * 4 * 5
+    rl, rows = O.reduced_layout(L, heads)
+    perm = np.zeros(rl.S, np.int32)
+    tc = np.zeros((rl.S + 127) // 128, np.uint8)
+    nv = h3.h3_layout_export(red, perm, tc)
+    assert nv == int(np.count_nonzero(rl.tags >= 0))
+    np.testing.assert_array_equal(perm, O.compaction_perm(rl.tags))
+    np.testing.assert_array_equal(tc, O.tile_classes(rl.tags))
+
+
+@pytest.mark.parametrize("r0,r1", [(1, 3), (0, 4), (2, 2)])
+def test_reduced_stack_small_amplified(r0, r1):
+    dims = SMALL_W
+    segs = [("text", 0, 41), ("video", (3, 4, 6), 0, 3), ("pad", 13), ("audio", 0, 57)]
+    L, target = _layout(segs)
+    ws_host = [amplified_weights(dims, 700 + i, std=0.05, table_std=0.2) for i in range(4)]
+    tmod = (np.random.default_rng(11).standard_normal((L.n_t, 6, dims.hidden)) * 0.2
+            ).astype(np.float32)
+    B = 2
+    xb = normal_bf16((B, L.S, dims.hidden), [12, 13], 1.0)
+    x, dl, red, dws = _run(dims, L, target, ws_host, tmod, xb, r0, r1)
+    got = host_f64(x)
+    pad = L.tags < 0
+    for b in range(B):
+        x0 = O.bf16_to_f64(xb[b])
+        ref = O.stack_forward_reduced(x0[None], lambda i: ws_host[i], 4, L, tmod, dims, target,
+                                      r0, r1)[0]
+        assert_close(got[b], ref, what=f"reduced stack x_out b={b}", storage_rounding=True)
+        assert_close(got[b, ~pad] - x0[~pad], ref[~pad] - x0[~pad], what="reduced stack update",
+                     mabs=np.inf)
+        np.testing.assert_array_equal(got[b, pad], x0[pad])
+    if r0 >= r1:  # no reduction: bit-identical to the plain stack
+        x2 = dev_bf16(xb)
+        ws_b = h3.h3_workspace_size(dl.dims, B, L.S)
+        ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+        h3.h3_stack_forward(dl.dims, [w.c for w in dws], dl.handle, dev_f32(tmod), x2, B, ws, ws_b)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host_bits(x2), host_bits(x))
+
+
+def test_reduced_stack_full_width():
+    dims = FULL_DIMS
+    segs = [("text", 0, 96), ("video", (4, 8, 16), 0, 4), ("pad", 30), ("audio", 0, 300)]
+    L, target = _layout(segs)
+    ws_host = [block_weights(dims, 8, i) for i in range(3)]
+    g = np.random.default_rng(21)
+    tmod = (g.standard_normal((L.n_t, 6, dims.hidden)) * 0.02).astype(np.float32)
+    xb = normal_bf16((1, L.S, dims.hidden), [14, 15], 1.0)
+    x, _, _, _ = _run(dims, L, target, ws_host, tmod, xb, 1, 2)
+    got = host_f64(x)[0]
+    x0 = O.bf16_to_f64(xb[0])
+    ref = O.stack_forward_reduced(x0[None], lambda i: ws_host[i], 3, L, tmod, dims, target, 1, 2)[0]
+    pad = L.tags < 0
+    assert_close(got, ref, what="full-width reduced stack x_out")
+    assert_close(got[~pad] - x0[~pad], ref[~pad] - x0[~pad], what="full-width reduced update",
+                 mabs=np.inf)

@@ -880,3 +880,138 @@ def test_denoiser_rows_permute_with_their_layout_and_padding_is_inert():
     vq, aq = run(Lq)
     np.testing.assert_array_equal(vq, vv)
     np.testing.assert_array_equal(aq, va)
+
+
+# ---------------------------------------------------------------- token reduction
+
+def test_reduction_pairs_by_hand():
+    """A (1, 2, 5) target grid: in each of the two h rows, w = (0, 1) and
+    (2, 3) pair and w = 4 stays single; a conditioning frame, text, audio and a
+    pair across different timesteps never pair."""
+    L = make_layout([("text", 0, 3), ("video", (2, 2, 5), 0, 2), ("audio", 0, 4)],
+                    timesteps="given", t_values=np.array([0.0, 0.5], np.float32),
+                    t_idx=np.zeros(27, np.int32))
+    target = (L.tags == 0) & (L.pos[:, 0] == 1)   # frame 1 is the target, frame 0 a reference
+    heads = O.reduction_pairs(L, target)
+    # rows: text 0..2, frame 0 at 3..12, frame 1 at 13..22 (h 0: 13..17, h 1: 18..22)
+    np.testing.assert_array_equal(heads, [13, 15, 18, 20])
+    red, rows = O.reduced_layout(L, heads)
+    assert red.S == 27 - 4
+    j = int(np.nonzero(rows[:, 0] == 13)[0][0])
+    assert rows[j, 1] == 14 and np.allclose(red.pos[j], [1, 0, 0.5])
+    L.t_idx[14] = 1  # the second row of the first pair moves to another timestep
+    np.testing.assert_array_equal(O.reduction_pairs(L, target), [15, 18, 20])
+    assert O.reduction_pairs(L, np.zeros(L.S, bool)).size == 0
+
+
+def test_merge_and_restore():
+    g = np.random.default_rng(3)
+    x = g.standard_normal((6, 4))
+    rows = np.array([[0, 1], [2, -1], [3, 4], [5, -1]])
+    m = O.merge_rows(x, rows)
+    np.testing.assert_allclose(m[0], 0.5 * (x[0] + x[1]))
+    np.testing.assert_array_equal(m[1], x[2])
+    # no change in the reduced rows restores the bypass exactly
+    np.testing.assert_allclose(O.restore_rows(x, m, rows), x, rtol=0, atol=1e-15)
+    # a change of a merged row reaches both rows of its pair
+    d = np.zeros_like(m)
+    d[2] = [1, 2, 3, 4]
+    out = O.restore_rows(x, m + d, rows)
+    np.testing.assert_allclose(out[3] - x[3], [1, 2, 3, 4], atol=1e-14)
+    np.testing.assert_allclose(out[4] - x[4], [1, 2, 3, 4], atol=1e-14)
+    np.testing.assert_allclose(np.delete(out, [3, 4], 0), np.delete(x, [3, 4], 0), atol=1e-15)
+
+
+def _reduction_case(seed=0):
+    segs = [("text", 0, 9), ("video", (3, 2, 6), 0, 3), ("pad", 5), ("audio", 0, 11)]
+    L0 = make_layout(segs, seed=[seed])
+    target = (L0.tags == 0) & (L0.pos[:, 0] >= 1)  # video frames 1, 2; frame 0 a reference
+    t_idx = (target | (L0.tags == 2)).astype(np.int32)
+    L = make_layout(segs, timesteps="given", t_values=np.array([0.0, 0.6], np.float32),
+                    t_idx=t_idx)
+    assert O.reduction_pairs(L, target).size == 12
+    ws = [_weights_big_gates(SMALL, 40 + i) for i in range(4)]
+    tmod = _tmod_random(L.n_t, SMALL.hidden, seed)
+    x = O.bf16_to_f64(f32_to_bf16_bits(np.random.default_rng([seed, 1]).standard_normal(
+        (1, L.S, SMALL.hidden)).astype(np.float32)))
+    return L, target, ws, tmod, x
+
+
+def test_reduced_stack_without_reduction_is_the_stack():
+    L, target, ws, tmod, x = _reduction_case(1)
+    full = O.stack_forward(x, lambda i: ws[i], 4, L, tmod, SMALL)
+    np.testing.assert_array_equal(
+        O.stack_forward_reduced(x, lambda i: ws[i], 4, L, tmod, SMALL, target, 2, 2), full)
+    # no target rows: every row maps to itself, and the restore x + (x_red - x)
+    # gives x_red up to the rounding of that sum
+    np.testing.assert_allclose(
+        O.stack_forward_reduced(x, lambda i: ws[i], 4, L, tmod, SMALL, np.zeros(L.S, bool), 1, 3),
+        full, rtol=1e-12, atol=1e-12)
+    red = O.stack_forward_reduced(x, lambda i: ws[i], 4, L, tmod, SMALL, target, 1, 3)
+    assert _rel(red, full) > 1e-3  # the reduction changes the result
+    pad = L.tags < 0
+    np.testing.assert_array_equal(red[0, pad], x[0, pad])
+
+
+def test_reduced_blocks_with_zero_gates_restore_the_bypass():
+    """Reduced blocks whose gates are all zero leave the merged rows unchanged, so
+    the restore gives back the bypass exactly, and the stack equals the full
+    stack without those blocks."""
+    import copy
+    L, target, ws, tmod, x = _reduction_case(2)
+    z = []
+    for w in ws:
+        w = copy.copy(w)
+        w.ada_table = np.array(w.ada_table, copy=True)
+        z.append(w)
+    for i in (1, 2):
+        z[i].ada_table[:, [2, 5]] = 0.0
+    tz = tmod.copy()
+    tz[:, [2, 5]] = 0.0
+    got = O.stack_forward_reduced(x, lambda i: z[i], 3, L, tz, SMALL, target, 1, 3)
+    ref = O.block_forward(x, z[0], L, tz, SMALL)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_reduced_stack_one_pair_by_hand():
+    """Two target rows that pair and nothing else: the reduced block sees one
+    row (a document of one key: its attention output is its own v), and the
+    restore adds that row's update to both rows."""
+    L = make_layout([("video", (1, 1, 2), 0, 1)], timesteps="given",
+                    t_values=np.array([0.5], np.float32), t_idx=np.zeros(2, np.int32))
+    target = np.ones(2, bool)
+    w = _weights_big_gates(SMALL, 9)
+    tmod = _tmod_random(1, SMALL.hidden, 9)
+    x = np.random.default_rng(4).standard_normal((1, 2, SMALL.hidden))
+    got = O.stack_forward_reduced(x, lambda i: w, 1, L, tmod, SMALL, target, 0, 1)
+    m = 0.5 * (x[0, 0] + x[0, 1])
+    Lm = make_layout([("video", (1, 1, 1), 0, 1)], timesteps="given",
+                     t_values=np.array([0.5], np.float32), t_idx=np.zeros(1, np.int32))
+    Lm.pos[0] = [0.0, 0.0, 0.5]
+    y = O.block_forward(m[None, None], w, Lm, tmod, SMALL)[0, 0]
+    np.testing.assert_allclose(got[0, 0], x[0, 0] + (y - m), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got[0, 1], x[0, 1] + (y - m), rtol=1e-12, atol=1e-12)
+
+
+def test_core_reuse_with_the_same_latents_is_the_full_forward():
+    """Reusing the core residual of a forward for the same latents gives that
+    forward's velocities (the residual is the stack's output minus its input);
+    with fresh latents only the projections and heads change."""
+    d, L, dw, blocks, video, audio, text = _denoiser_case(4)
+    res = np.zeros((L.S, d.hidden))
+    vv, va = O.denoiser_forward(video, audio, text, dw, lambda i: blocks[i], 2, L, d, 1e-5,
+                                core_residual=res)
+    assert np.linalg.norm(res) > 0
+    rv, ra = O.denoiser_forward(video, audio, text, dw, lambda i: blocks[i], 2, L, d, 1e-5,
+                                core_residual=res, reuse=True)
+    np.testing.assert_allclose(rv, vv, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ra, va, rtol=1e-12, atol=1e-12)
+    # fresh latents: head(norm_out(projection + residual)), rebuilt by hand
+    v2 = video * 0.5 + 0.1
+    rv2, _ = O.denoiser_forward(v2, audio, text, dw, lambda i: blocks[i], 2, L, d, 1e-5,
+                                core_residual=res, reuse=True)
+    tmo = O.output_modulation(L.timestep, dw.w_t1, dw.w_t2, dw.w_out, d.freq_dim, d.hidden)
+    m = np.asarray(dw.out_table)[0][None] + tmo[L.t_idx[L.video_idx]]
+    xr = v2 @ np.asarray(dw.w_patch_video).T + res[L.video_idx]
+    np.testing.assert_allclose(rv2, O.output_head(xr, m[:, 0], m[:, 1], dw.w_head_video, 1e-5),
+                               rtol=1e-12, atol=1e-12)
