@@ -36,26 +36,8 @@ __device__ __forceinline__ void load8(const float* p, float* v) {
 // the mean is far from zero); pass 2 reads x again (L1 / L2) together with the
 // row's modulation and writes h. Nothing is held across the passes, so the
 // kernel runs with few registers and many rows in flight per SM.
-// Variants under measurement: bit 0 prefetches the row's modulation rows of
-// tmod into L2 during the statistics pass; bit 1 caps registers so that more
-// rows are in flight per SM; bit 2 unrolls the second pass further.
-#ifndef H3_NORM_VARIANT
-#define H3_NORM_VARIANT 0
-#endif
-#if H3_NORM_VARIANT & 2
-#define H3_NORM_BOUNDS __launch_bounds__(256, 6)
-#else
-#define H3_NORM_BOUNDS __launch_bounds__(256)
-#endif
-
-#if H3_NORM_VARIANT & 1
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-#endif
-
 template <typename XT>
-__global__ void H3_NORM_BOUNDS k_norm_modulate(
+__global__ void __launch_bounds__(256) k_norm_modulate(
     int rows, int S, int H, int chunk_shift, int chunk_scale, float eps,
     const XT* __restrict__ x, const int32_t* __restrict__ tags,
     const int32_t* __restrict__ t_idx, const float* __restrict__ table,
@@ -80,17 +62,6 @@ __global__ void H3_NORM_BOUNDS k_norm_modulate(
     c = __shfl_sync(0xffffffffu, v[0], 0);
   }
   float sum = 0.f, sq = 0.f;
-#if H3_NORM_VARIANT & 1
-  {
-    // 128-byte lines of the shift and scale rows of tmod: 2H fp32 = H / 16 lines
-    const char* m0 = reinterpret_cast<const char*>(tmod + ((size_t)ti * 6 + chunk_shift) * H);
-    const char* m1 = reinterpret_cast<const char*>(tmod + ((size_t)ti * 6 + chunk_scale) * H);
-    for (int l = lane; l < H / 32; l += 32) {
-      prefetch_l2(m0 + 128 * l);
-      prefetch_l2(m1 + 128 * l);
-    }
-  }
-#endif
 #pragma unroll 4
   for (int i = 0; i < nv; ++i) {
     float v[8];
@@ -115,11 +86,7 @@ __global__ void H3_NORM_BOUNDS k_norm_modulate(
   const float4* sc_t = reinterpret_cast<const float4*>(table + ((size_t)tag * 6 + chunk_scale) * H);
   const float4* sh_m = reinterpret_cast<const float4*>(tmod + ((size_t)ti * 6 + chunk_shift) * H);
   const float4* sc_m = reinterpret_cast<const float4*>(tmod + ((size_t)ti * 6 + chunk_scale) * H);
-#if H3_NORM_VARIANT & 4
-#pragma unroll 4
-#else
 #pragma unroll 2
-#endif
   for (int i = 0; i < nv; ++i) {
     const int e4 = 2 * (lane + 32 * i);  // float4 index of the first of the 8 elements
     float xs[8];
