@@ -24,11 +24,8 @@
 // guarantees PV_i(j) is complete: the softmax may then rescale O_i in place.
 // O is rescaled only when a row's running max grows by more than 2^8 (lazy
 // rescale), decided per warp because TMEM loads / stores are warp-collective.
-// After the first key tile the exponentials run against the running max while
-// the tile's max is taken in the same pass; a tile that raises it beyond the
-// threshold redoes its first half (the result is that of max-first).
-// exp2 runs on the MUFU for three quarters of the key pairs and as a
-// polynomial on the FMA pipe for every fourth pair, to keep both pipes busy.
+// exp2 runs on the MUFU for most key pairs and as a polynomial on the FMA pipe
+// for every sixth pair, to keep both pipes busy.
 // P is handed to the MMA warp in two halves (keys 0..63, then 64..127), so the
 // first half of P V runs while the second half's exponentials are computed.
 //
@@ -48,8 +45,10 @@ constexpr int HALF = 128 * 64 * 2;  // one 128-row x 64-column bf16 half tile: 1
 constexpr int TILE_BYTES = 2 * HALF;
 constexpr int NUM_THREADS = 384;
 // Registers per thread after the split; launched at 65536 / 384 -> 168 each:
-// 2 * 128 * kSoftmaxRegs + 128 * kControlRegs must not exceed 384 * 168.
-constexpr uint32_t kSoftmaxRegs = 224, kControlRegs = 56;
+// 2 * 128 * kSoftmaxRegs + 128 * kControlRegs must not exceed 384 * 168. With
+// 216 / 72 neither the softmax nor the producer / MMA loops spill (224 / 56
+// spills in the control warps, 208 / 88 in the softmax warps).
+constexpr uint32_t kSoftmaxRegs = 216, kControlRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= 384 * 168, "register split");
 constexpr int TMEM_COLS = 512;
 constexpr float kLazyRescale = 8.0f;  // log2 units
@@ -121,12 +120,14 @@ __device__ __forceinline__ void exp2_poly2(uint64_t x2, float& p0, float& p1) {
   p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-// Which key pairs of a 64-key half take the FMA-pipe exp2: every kPolyEvery-th
-// pair, spread among the MUFU pairs so that both pipes work at the same time.
-#ifndef H3_ATTN_POLY_EVERY
-#define H3_ATTN_POLY_EVERY 4
+// Which key pairs of a 64-key half take the FMA-pipe exp2 (bit e of the mask
+// for pair e), spread among the MUFU pairs so that both pipes work at the same
+// time. Default: every sixth pair (pairs 5, 11, 17, 23, 29: 16 %), the fastest
+// of the splits measured (50, 40, 33, 25, 16, 12.5 and 0 %).
+#ifndef H3_ATTN_POLY_MASK
+#define H3_ATTN_POLY_MASK 0x20820820u
 #endif
-constexpr int kPolyEvery = H3_ATTN_POLY_EVERY;
+constexpr uint32_t kPolyMask = H3_ATTN_POLY_MASK;
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
@@ -362,115 +363,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!((bits >> e) & 1u)) sc[32 * w + e] = -INFINITY;
         }
       }
+      // row max: 8 independent partial maxima
+      float pm[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) pm[k] = max3(sc[2 * k], sc[2 * k + 1], sc[16 + 2 * k]);
+#pragma unroll
+      for (int e = 32; e < 128; e += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pm[k] = max3(pm[k], sc[e + 2 * k], sc[e + 2 * k + 1]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) pm[k] = fmaxf(pm[k], sc[16 + 2 * k + 1]);
+      float mx = max3(max3(pm[0], pm[1], pm[2]), max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+      mx *= scale_log2;
+      // O_i is stable here: the commit that signalled S_i(j) follows PV_i(j-1).
+      const bool need = mx > m_run + kLazyRescale;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = need ? mx : m_run;
+        if (j > 0) {
+          const float alpha = exp2_mufu(m_run - m_new);
+          l_run *= alpha;
+          uint32_t rr[32];
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            tmem_ld32(o_col + 32 * c, rr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            tmem_st32(o_col + 32 * c, rr);
+          }
+        }
+        m_run = m_new;
+      }
       // P = 2^(s * scale - m), written as packed bf16 pairs over S columns
       // already held in registers: keys 0..63, then keys 64..127, each half
       // signalled to the MMA warp as soon as it is stored (one arrival per warp,
-      // after the warp's stores are complete). Every kPolyEvery-th key pair
-      // takes the FMA-pipe exp2, the others the MUFU.
+      // after the warp's stores are complete). The key pairs in kPolyMask take
+      // the FMA-pipe exp2, the others the MUFU.
+      const uint64_t negm2 = f2_pack(-m_run, -m_run);
       uint64_t sum2[4] = {0, 0, 0, 0};
-      uint32_t pk[32];
-      auto exp_pair = [&](uint64_t x2, float& p0, float& p1, int e) {
-        if (e % kPolyEvery == kPolyEvery - 1) {
-          exp2_poly2(x2, p0, p1);
-        } else {
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          p0 = exp2_mufu(x0);
-          p1 = exp2_mufu(x1);
-        }
-      };
-      auto exp_half = [&](int h, uint64_t negm2) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int key = 64 * h + 2 * e;
           const uint64_t x2 = f2_fma(f2_pack(sc[key], sc[key + 1]), scale2, negm2);
           float p0, p1;
-          exp_pair(x2, p0, p1, e);
+          if ((kPolyMask >> e) & 1u) {
+            exp2_poly2(x2, p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = exp2_mufu(x0);
+            p1 = exp2_mufu(x1);
+          }
           sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
-      };
-      auto store_signal = [&](int h) {
         tmem_st32(s_col + 32 * h, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(h == 0 ? &bars->p_half[i] : &bars->p_full[i]);
-      };
-      // O and l take the factor 2^(m_run - m_new) when a row's reference grows.
-      // O_i is stable here: the commit that signalled S_i(j) follows PV_i(j-1).
-      auto rescale = [&](float m_new) {
-        const float alpha = exp2_mufu(m_run - m_new);
-        l_run *= alpha;
-        uint32_t rr[32];
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(o_col + 32 * c, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-          tmem_st32(o_col + 32 * c, rr);
-        }
-      };
-      if (j > 0) {
-        // The exps of keys 0..63 run against the running max m_run; the tile's
-        // row max relative to m_run comes out of the same loop (those x values,
-        // and the raw scores of keys 64..127 interleaved). Only when it exceeds
-        // the lazy-rescale threshold (rare after the first tiles) does the row
-        // take a new reference, rescale O and l, and redo keys 0..63: the
-        // result is the same as computing the max first.
-        uint64_t negm2 = f2_pack(-m_run, -m_run);
-        float xm[4], sm[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) xm[k] = sm[k] = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int key = 2 * e;
-          const uint64_t x2 = f2_fma(f2_pack(sc[key], sc[key + 1]), scale2, negm2);
-          float x0, x1, p0, p1;
-          f2_unpack(x2, x0, x1);
-          xm[e & 3] = max3(xm[e & 3], x0, x1);
-          sm[e & 3] = max3(sm[e & 3], sc[64 + key], sc[64 + key + 1]);
-          exp_pair(x2, p0, p1, e);
-          sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        const float rel =
-            fmaxf(fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3])),
-                  fmaf(fmaxf(fmaxf(sm[0], sm[1]), fmaxf(sm[2], sm[3])), scale_log2, -m_run));
-        const bool need = rel > kLazyRescale;
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = need ? m_run + rel : m_run;
-          rescale(m_new);
-          m_run = m_new;
-          negm2 = f2_pack(-m_run, -m_run);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) sum2[k] = 0;
-          exp_half(0, negm2);
-        }
-        store_signal(0);
-        exp_half(1, negm2);
-        store_signal(1);
-      } else {
-        // first tile: the row max first (8 independent partial maxima)
-        float pm[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) pm[k] = max3(sc[2 * k], sc[2 * k + 1], sc[16 + 2 * k]);
-#pragma unroll
-        for (int e = 32; e < 128; e += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) pm[k] = max3(pm[k], sc[e + 2 * k], sc[e + 2 * k + 1]);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) pm[k] = fmaxf(pm[k], sc[16 + 2 * k + 1]);
-        const float mx =
-            max3(max3(pm[0], pm[1], pm[2]), max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])) *
-            scale_log2;
-        m_run = mx > m_run + kLazyRescale ? mx : m_run;
-        const uint64_t negm2 = f2_pack(-m_run, -m_run);
-        exp_half(0, negm2);
-        store_signal(0);
-        exp_half(1, negm2);
-        store_signal(1);
       }
       float a0, a1, b0, b1;
       f2_unpack(f2_add(sum2[0], sum2[1]), a0, a1);

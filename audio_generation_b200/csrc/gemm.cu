@@ -59,18 +59,8 @@ constexpr int NUM_THREADS = 192;
 static __device__ int g_fault_skip_loads;
 #endif
 
-// L2 policies: 0 none; 1 weight (B) tiles loaded evict_last; 2 also the
-// epilogue's bf16 output stores evict_first, so the output stream does not
-// push the N-group's weight tiles out of L2.
-#ifndef H3_GEMM_L2_HINTS
-#define H3_GEMM_L2_HINTS 0
-#endif
-
 __device__ __forceinline__ void store_bf16x32(void* dst, const float* y) {
   uint4* d = reinterpret_cast<uint4*>(dst);
-#if H3_GEMM_L2_HINTS >= 2
-  const uint64_t pol = l2_policy_evict_first();
-#endif
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint4 u;
@@ -78,11 +68,7 @@ __device__ __forceinline__ void store_bf16x32(void* dst, const float* y) {
     u.y = pack_bf16x2(y[8 * q + 2], y[8 * q + 3]);
     u.z = pack_bf16x2(y[8 * q + 4], y[8 * q + 5]);
     u.w = pack_bf16x2(y[8 * q + 6], y[8 * q + 7]);
-#if H3_GEMM_L2_HINTS >= 2
-    st_global_v4_hint(d + q, u, pol);
-#else
     d[q] = u;
-#endif
   }
 }
 
@@ -321,9 +307,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       uint32_t n = 0;
       bool ok = true;
-#if H3_GEMM_L2_HINTS >= 1
-      const uint64_t b_policy = l2_policy_evict_last();
-#endif
 #ifdef H3_FAULT_INJECTION
       if (*(volatile int*)&g_fault_skip_loads) ok = false;
 #endif
@@ -340,12 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           uint8_t* sa = smem + s * P_STAGE;
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE);
           tma_load_2d_pair(sa, &tmA, at(&full[s], 0), kb * BK, m0);
-#if H3_GEMM_L2_HINTS >= 1
-          tma_load_2d_pair_hint(sa + A_STAGE, &tmB, at(&full[s], 0), kb * BK,
-                                n0 + (BN / 2) * rank, b_policy);
-#else
           tma_load_2d_pair(sa + A_STAGE, &tmB, at(&full[s], 0), kb * BK, n0 + (BN / 2) * rank);
-#endif
           ++n;
         }
       }

@@ -475,9 +475,15 @@ def run_gpu(args, world, rank, local):
             per[name] += evs[r][i].elapsed_time(evs[r][i + 1]) / reps
     work = kernel_work(dims, V)
     peaks = load_peaks()
-    # Kernels timed right after a seconds-long run of steps run at the power-capped
-    # clock: their tensor peak is the sustained cuBLAS figure, else the burst one.
-    long_run = args.steps * ms_per_step >= 1000.0
+    # Kernels timed inside and right after a run of block steps: when the SM
+    # clock sampled over the timed steps sits below 90 % of its maximum (the
+    # board at its power cap) or the steps ran for a second or more, the
+    # kernels ran in the sustained power state and their tensor peak is the
+    # sustained cuBLAS figure; otherwise the burst one. Both fractions are given.
+    clocks = clk.summary()
+    capped = (clocks.get("sm_mhz") is not None and clocks.get("sm_max_mhz")
+              and clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"])
+    long_run = args.steps * ms_per_step >= 1000.0 or bool(capped)
     tc_peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
     peak_kind = "sustained" if long_run else "burst"
     dom = max(per, key=lambda n: per[n])
@@ -499,7 +505,6 @@ def run_gpu(args, world, rank, local):
             kernels[n] = {"ms": round(per[n], 4), "gbs": round(amt / t / 1e9, 1),
                           "frac_of_peak": round(amt / t / 1e9 / peaks["hbm_gbs"], 3)}
     flops = block_flops(dims, V)
-    clocks = clk.summary()
     del hbuf, q, k, v, o, gbuf
     masked = None if args.no_masked else masked_attention(h3, d, dims, device, stream, peaks)
     line = {
@@ -518,6 +523,9 @@ def run_gpu(args, world, rank, local):
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
                      "unit": unit, "frac": achieved / peak, "traffic": measured_traffic(dom, cfg),
                      "peak_kind": peak_kind if bound == "tensor" else "copy",
+                     "frac_of_burst": (achieved / peaks["bf16_tflops"] if bound == "tensor"
+                                       else achieved / peak),
+                     "clock_sm_mhz": clocks.get("sm_mhz"),
                      "algorithmic_bytes": kernel_bytes(dims, V)[dom]},
         "kernels": kernels,
         "attention_masked": masked,
@@ -573,7 +581,8 @@ def masked_attention(h3, d, dims, device, stream, peaks, reps=10):
     tf = 4.0 * dims.heads * dims.head_dim * float(V) ** 2 / (ms * 1e-3) / 1e12
     return {"workload": WORKLOADS[MASKED_CFG], "S": S, "valid_rows": V, "launches": reps,
             "ms": round(ms, 4), "tflops_valid": round(tf, 1),
-            "frac_of_peak": round(tf / peaks["bf16_tflops"], 3), "peak_kind": "burst"}
+            "frac_of_peak": round(tf / peaks["bf16_tflops"], 3), "peak_kind": "burst",
+            "frac_of_sustained_peak": round(tf / peaks["bf16_tflops_sustained"], 3)}
 
 
 STACK_CFG = 5

@@ -106,5 +106,10 @@ def test_reduced_stack_full_width():
     ref = O.stack_forward_reduced(x0[None], lambda i: ws_host[i], 3, L, tmod, dims, target, 1, 2)[0]
     pad = L.tags < 0
     assert_close(got, ref, what="full-width reduced stack x_out")
-    assert_close(got[~pad] - x0[~pad], ref[~pad] - x0[~pad], what="full-width reduced update",
+    # The stack rounds its fp32 stream to bf16 once, when it scatters the rows
+    # back; at these gates that single rounding is ~1 % of the three blocks'
+    # update, so the update is compared with the float64 result rounded at the
+    # same point (the same comparison gives 1.1e-2 for the plain stack without it).
+    ref_q = O.round_bf16(ref)
+    assert_close(got[~pad] - x0[~pad], ref_q[~pad] - x0[~pad], what="full-width reduced update",
                  mabs=np.inf)
