@@ -98,14 +98,26 @@ h3_status check_weights(const h3_block_weights* w) {
 
 // One block over the rows described by `L` (full or compacted view), in place on
 // x: bf16 for h3_block_forward, fp32 (x_f32) for the stack's residual stream.
+// 8-bit operands of the QKV and W1 || W3 GEMMs (null: the bf16 block). codes
+// [M, H] bytes and scales [M] are workspace for the activation rows.
+struct E4m3Operands {
+  const h3_block_weights_e4m3* w = nullptr;
+  void* codes = nullptr;
+  float* scales = nullptr;
+};
+
 h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutView& L,
                     const float* tmod, void* x, bool x_f32, int B, const Workspace& ws,
-                    cudaStream_t st) {
+                    cudaStream_t st, const E4m3Operands& q8 = E4m3Operands()) {
   const int M = B * L.S;
   if (M == 0) return H3_OK;
   const int H = d.hidden, A = d.heads * d.head_dim, Fd = d.ffn;
-  H3_CUDA(launch_norm_modulate(L, B, H, 0, 1, d.norm_eps, x, x_f32, w.ada_table, tmod, ws.h,
-                               st));
+  if (q8.w)
+    H3_CUDA(launch_norm_modulate_e4m3(L, B, H, 0, 1, d.norm_eps, x, x_f32, w.ada_table, tmod,
+                                      q8.codes, q8.scales, st));
+  else
+    H3_CUDA(launch_norm_modulate(L, B, H, 0, 1, d.norm_eps, x, x_f32, w.ada_table, tmod, ws.h,
+                                 st));
   GemmEpiArgs e;
   e.L = L;
   e.B = B;
@@ -116,7 +128,13 @@ h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutVie
   e.q_norm = w.q_norm;
   e.k_norm = w.k_norm;
   e.qk_eps = d.qk_norm_eps;
-  H3_CUDA(launch_gemm(EPI_QKV, M, 3 * A, H, ws.h, w.w_qkv, e, st));
+  if (q8.w) {
+    e.a_scale = q8.scales;
+    e.b_scale = q8.w->w_qkv_scales;
+    H3_CUDA(launch_gemm_e4m3(EPI_QKV, M, 3 * A, H, q8.codes, q8.w->w_qkv_codes, e, st));
+  } else {
+    H3_CUDA(launch_gemm(EPI_QKV, M, 3 * A, H, ws.h, w.w_qkv, e, st));
+  }
   H3_CUDA(launch_attention(L, B, d.heads, ws.q, ws.k, ws.v, ws.o, st));
   GemmEpiArgs r;
   r.L = L;
@@ -127,12 +145,20 @@ h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutVie
   r.gate_chunk = 2;
   const int resid = x_f32 ? EPI_RESID_F32 : EPI_RESID;
   H3_CUDA(launch_gemm(resid, M, H, A, ws.o, w.w_o, r, st));
-  H3_CUDA(launch_norm_modulate(L, B, H, 3, 4, d.norm_eps, x, x_f32, w.ada_table, tmod, ws.h,
-                               st));
   GemmEpiArgs sg;
   sg.L = L;
   sg.out = ws.g;
-  H3_CUDA(launch_gemm(EPI_SWIGLU, M, 2 * Fd, H, ws.h, w.w13, sg, st));
+  if (q8.w) {
+    H3_CUDA(launch_norm_modulate_e4m3(L, B, H, 3, 4, d.norm_eps, x, x_f32, w.ada_table, tmod,
+                                      q8.codes, q8.scales, st));
+    sg.a_scale = q8.scales;
+    sg.b_scale = q8.w->w13_scales;
+    H3_CUDA(launch_gemm_e4m3(EPI_SWIGLU, M, 2 * Fd, H, q8.codes, q8.w->w13_codes, sg, st));
+  } else {
+    H3_CUDA(launch_norm_modulate(L, B, H, 3, 4, d.norm_eps, x, x_f32, w.ada_table, tmod, ws.h,
+                                 st));
+    H3_CUDA(launch_gemm(EPI_SWIGLU, M, 2 * Fd, H, ws.h, w.w13, sg, st));
+  }
   r.gate_chunk = 5;
   H3_CUDA(launch_gemm(resid, M, H, Fd, ws.g, w.w2, r, st));
   return H3_OK;
@@ -756,6 +782,53 @@ h3_status h3_stack_forward_reduced(const h3_dims* dims, const h3_block_weights* 
     H3_TRY(run_block(d, weights[i], full->compact_view(), tmod, xc, true, B, w, st));
   H3_CUDA(launch_permute_rows_convert(B, V, full->S, H, full->perm, xc, x, false, st));
   return H3_OK;
+}
+
+}  // extern "C"
+
+// ---- 8-bit QKV and W1 || W3 GEMM inputs ----
+
+extern "C" {
+
+h3_status h3_quantize_e4m3_rows(const void* w, int rows, int K, void* codes, float* scales,
+                                h3_stream_t stream) {
+  if (rows < 0 || K <= 0 || (rows > 0 && (!w || !codes || !scales))) return H3_ERR_ARG;
+  if (K % 16 != 0) return H3_ERR_SHAPE;
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(scales)) return H3_ERR_ALIGN;
+  H3_CUDA(launch_quantize_rows_e4m3(rows, K, w, codes, scales, as_stream(stream)));
+  return H3_OK;
+}
+
+size_t h3_workspace_size_e4m3(const h3_dims* dims, int B, int S) {
+  if (check_dims(dims) != H3_OK || B < 0 || S < 0) return 0;
+  const size_t rows = (size_t)B * S;
+  return ws_parts(*dims, B, S, nullptr, nullptr) + align256(rows * dims->hidden) +
+         align256(rows * 4);
+}
+
+h3_status h3_block_forward_e4m3(const h3_dims* dims, const h3_block_weights* weights,
+                                const h3_block_weights_e4m3* w8, h3_layout_t L,
+                                const float* tmod, void* x, int B, void* ws, size_t ws_bytes,
+                                h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !tmod || !x || !ws || !w8) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
+  H3_TRY(check_weights(weights));
+  if (!w8->w_qkv_codes || !w8->w_qkv_scales || !w8->w13_codes || !w8->w13_scales)
+    return H3_ERR_ARG;
+  if (!aligned16(w8->w_qkv_codes) || !aligned16(w8->w_qkv_scales) || !aligned16(w8->w13_codes) ||
+      !aligned16(w8->w13_scales) || !aligned16(tmod) || !aligned16(x) || !aligned16(ws))
+    return H3_ERR_ALIGN;
+  if (dims->hidden % 128 != 0) return H3_ERR_SHAPE;
+  if (ws_bytes < h3_workspace_size_e4m3(dims, B, L->S)) return H3_ERR_WORKSPACE;
+  Workspace w;
+  const size_t base = ws_parts(*dims, B, L->S, &w, ws);
+  E4m3Operands q8;
+  q8.w = w8;
+  q8.codes = static_cast<uint8_t*>(ws) + base;
+  q8.scales = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + base +
+                                       align256((size_t)B * L->S * dims->hidden));
+  return run_block(*dims, *weights, L->view(), tmod, x, false, B, w, as_stream(stream), q8);
 }
 
 }  // extern "C"

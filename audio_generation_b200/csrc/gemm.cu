@@ -38,6 +38,9 @@
 //   EPI_SWIGLU W1 / W3 interleaved in 128-row blocks: g = SiLU(a) * b.
 //   EPI_STORE  plain bf16 store (the GEMM core on its own).
 //   EPI_F32    plain fp32 store (the prologue's split-operand GEMMs).
+// The QKV and SwiGLU epilogues also come in an e4m3 form (kind::f8f6f4 MMAs
+// over 128-element K stages of 8-bit codes), whose accumulator is multiplied
+// by the row's activation scale and the column's weight scale first.
 #include "host_util.cuh"
 #include "internal.cuh"
 #include "sm100.cuh"
@@ -92,12 +95,32 @@ __device__ __forceinline__ void ld_acc(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// The accumulator of an e4m3 GEMM times the row's activation scale and each
+// column's weight scale (a bf16 GEMM's accumulator as it is).
+template <bool F8>
+__device__ __forceinline__ void ld_acc_s(uint32_t taddr, float* v, float sa, const float* sw) {
+  ld_acc(taddr, v);
+  if constexpr (F8) {
+    const float4* w4 = reinterpret_cast<const float4*>(sw);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 w = __ldg(w4 + q);
+      v[4 * q] *= sa * w.x;
+      v[4 * q + 1] *= sa * w.y;
+      v[4 * q + 2] *= sa * w.z;
+      v[4 * q + 3] *= sa * w.w;
+    }
+  }
+}
+
 // Epilogue for one 128 x 256 accumulator tile. Every lane of the warp executes
 // the TMEM loads (they are warp-collective); stores are predicated per row.
-template <int EPI, int BN>
+template <int EPI, int BN, bool F8>
 __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int M, int N,
                                               const GemmEpiArgs& e) {
   const bool row_ok = m < M;
+  [[maybe_unused]] float sa = 1.f;
+  if constexpr (F8) sa = row_ok ? e.a_scale[m] : 0.f;
   if constexpr (EPI == EPI_STORE) {
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(e.out);
 #pragma unroll 1
@@ -125,8 +148,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       float a[32], b[32];
-      ld_acc(taddr + 32 * c, a);
-      ld_acc(taddr + 128 + 32 * c, b);
+      ld_acc_s<F8>(taddr + 32 * c, a, sa, e.b_scale + n0 + 32 * c);
+      ld_acc_s<F8>(taddr + 128 + 32 * c, b, sa, e.b_scale + n0 + 128 + 32 * c);
 #pragma unroll
       for (int i = 0; i < 32; ++i) a[i] = a[i] / (1.f + __expf(-a[i])) * b[i];
       if (row_ok) store_bf16x32(out + (size_t)m * ldo + n0 / 2 + 32 * c, a);
@@ -188,11 +211,12 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
       __nv_bfloat16* dst =
           reinterpret_cast<__nv_bfloat16*>(kind == 0 ? e.q : (kind == 1 ? e.k : e.v)) +
           (((size_t)b * e.NH + head) * S + s) * 128;
+      const float* sw = e.b_scale + n0 + 128 * su;
       if (kind == 2) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float v[32];
-          ld_acc(tbase + 32 * c, v);
+          ld_acc_s<F8>(tbase + 32 * c, v, sa, sw + 32 * c);
           if (row_ok) store_bf16x32(dst + 32 * c, v);
         }
         continue;
@@ -201,7 +225,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float v[32];
-        ld_acc(tbase + 32 * c, v);
+        ld_acc_s<F8>(tbase + 32 * c, v, sa, sw + 32 * c);
 #pragma unroll
         for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
       }
@@ -211,7 +235,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float v[32], w[32];
-        ld_acc(tbase + 32 * c, v);
+        ld_acc_s<F8>(tbase + 32 * c, v, sa, sw + 32 * c);
         load_bf16x32(nw + 32 * c, w);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = v[i] * rstd * w[i];
@@ -250,7 +274,7 @@ constexpr int p_stage() { return (BM + BN / 2) * BK * 2; }
 template <int BN>
 constexpr int p_smem_bytes() { return PNST * p_stage<BN>() + 1024 + 256; }
 
-template <int EPI, int BN>
+template <int EPI, int BN, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 int M, int N, int K, int group_n, const GemmEpiArgs e) {
@@ -272,7 +296,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   const int tiles_m = (M + 2 * BM - 1) / (2 * BM), tiles_n = N / BN;
-  const int T = tiles_m * tiles_n, kb_n = K / BK;
+  // K elements per stage: 64 bf16 or 128 e4m3 (128 bytes either way)
+  constexpr int BKE = F8 ? 2 * BK : BK;
+  const int T = tiles_m * tiles_n, kb_n = K / BKE;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < PNST; ++s) {
@@ -322,8 +348,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           }
           uint8_t* sa = smem + s * P_STAGE;
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE);
-          tma_load_2d_pair(sa, &tmA, at(&full[s], 0), kb * BK, m0);
-          tma_load_2d_pair(sa + A_STAGE, &tmB, at(&full[s], 0), kb * BK, n0 + (BN / 2) * rank);
+          tma_load_2d_pair(sa, &tmA, at(&full[s], 0), kb * BKE, m0);
+          tma_load_2d_pair(sa + A_STAGE, &tmB, at(&full[s], 0), kb * BKE, n0 + (BN / 2) * rank);
           ++n;
         }
       }
@@ -334,7 +360,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     if (leader) {  // the whole warp runs the loop; one elected lane issues
-      constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, false, false);
+      constexpr uint32_t idesc =
+          F8 ? idesc_e4m3_f32(2 * BM, BN) : idesc_bf16_f32(2 * BM, BN, false, false);
       constexpr uint32_t hi = sdesc_hi_sw128(1024);
       const uint32_t base_lo = sdesc_lo(smem_u32(smem), 16);
       uint32_t n = 0, it = 0;
@@ -354,9 +381,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const uint32_t a_lo = base_lo + s * (P_STAGE >> 4);
           const uint32_t b_lo = a_lo + (A_STAGE >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_ss_w_pair_elect(d, a_lo + 2 * k, hi, b_lo + 2 * k, hi, idesc,
-                                 (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < BK / 16; ++k) {  // 32 bytes of K per instruction
+            if constexpr (F8)
+              umma_ss_w_pair_elect_f8(d, a_lo + 2 * k, hi, b_lo + 2 * k, hi, idesc,
+                                      (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_ss_w_pair_elect(d, a_lo + 2 * k, hi, b_lo + 2 * k, hi, idesc,
+                                   (kb | k) != 0 ? 1u : 0u);
+          }
           umma_commit_pair_elect(at(&empty[s], 0));
           umma_commit_pair_elect(at(&empty[s], 1));
           ++n;
@@ -381,7 +413,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       tile_coords<BN>(t, tiles_m, tiles_n, group_n, m0, n0);
       m0 = 2 * m0 + BM * rank;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-      epilogue_tile<EPI, BN>(taddr, m0 + row_local, n0, M, N, e);
+      epilogue_tile<EPI, BN, F8>(taddr, m0 + row_local, n0, M, N, e);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty1 : tempty0);
@@ -396,30 +428,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int EPI, int BN>
+template <int EPI, int BN, bool F8 = false>
 cudaError_t run(int M, int N, int K, const void* A, const void* Bm, const GemmEpiArgs& e,
                 cudaStream_t st) {
   constexpr int P_SMEM_BYTES = p_smem_bytes<BN>();
-  cudaError_t err = cudaFuncSetAttribute(k_gemm_pair<EPI, BN>,
+  cudaError_t err = cudaFuncSetAttribute(k_gemm_pair<EPI, BN, F8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          P_SMEM_BYTES);
   if (err != cudaSuccess) return err;
   CUtensorMap ta, tb;
-  const uint64_t da[2] = {(uint64_t)K, (uint64_t)M}, sa[1] = {(uint64_t)K * 2};
-  const uint32_t ba[2] = {BK, BM};
-  const uint64_t db[2] = {(uint64_t)K, (uint64_t)N}, sb[1] = {(uint64_t)K * 2};
-  const uint32_t bb[2] = {BK, BN / 2};  // each CTA of the pair loads half of the tile's B rows
-  if (!make_tmap_bf16(&ta, A, 2, da, sa, ba) || !make_tmap_bf16(&tb, Bm, 2, db, sb, bb))
+  constexpr uint64_t esz = F8 ? 1 : 2;
+  constexpr uint32_t bke = F8 ? 2 * BK : BK;  // 128 bytes of K per box row
+  const CUtensorMapDataType type =
+      F8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t da[2] = {(uint64_t)K, (uint64_t)M}, sa[1] = {(uint64_t)K * esz};
+  const uint32_t ba[2] = {bke, BM};
+  const uint64_t db[2] = {(uint64_t)K, (uint64_t)N}, sb[1] = {(uint64_t)K * esz};
+  const uint32_t bb[2] = {bke, BN / 2};  // each CTA of the pair loads half of the tile's B rows
+  if (!make_tmap(&ta, A, type, 2, da, sa, ba) || !make_tmap(&tb, Bm, type, 2, db, sb, bb))
     return cudaErrorInvalidValue;
   const int T = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
   const int max_pairs = num_sms() / 2;
   const int n_pairs = T < max_pairs ? T : max_pairs;
   // Weight tiles kept L2-resident per group: about 48 MB of B.
-  const long long b_tile_bytes = (long long)BN * K * 2;
+  const long long b_tile_bytes = (long long)BN * K * esz;
   int group_n = (int)((48ll << 20) / b_tile_bytes);
   if (group_n < 1) group_n = 1;
   if (group_n > N / BN) group_n = N / BN;
-  k_gemm_pair<EPI, BN><<<2 * n_pairs, NUM_THREADS, P_SMEM_BYTES, st>>>(ta, tb, M, N, K, group_n, e);
+  k_gemm_pair<EPI, BN, F8><<<2 * n_pairs, NUM_THREADS, P_SMEM_BYTES, st>>>(ta, tb, M, N, K,
+                                                                          group_n, e);
   return cudaGetLastError();
 }
 
@@ -432,6 +469,18 @@ long long wave_cost(int M, int N, int bn) {
 }
 
 }  // namespace
+
+cudaError_t launch_gemm_e4m3(int epi, int M, int N, int K, const void* A, const void* Bm,
+                             const GemmEpiArgs& e, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  if (K % (2 * BK) != 0 || K == 0 || N % 256 != 0 || !e.a_scale || !e.b_scale)
+    return cudaErrorInvalidValue;
+  switch (epi) {
+    case EPI_QKV: return run<EPI_QKV, 256, true>(M, N, K, A, Bm, e, st);
+    case EPI_SWIGLU: return run<EPI_SWIGLU, 256, true>(M, N, K, A, Bm, e, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void* Bm,
                         const GemmEpiArgs& e, cudaStream_t st) {

@@ -82,6 +82,11 @@ h3_status symbol_address(SymbolAddressCache& cache, cudaError_t (*lookup)(void**
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_tmap(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, dims, strides_bytes, box);
+}
+
+bool make_tmap(CUtensorMap* map, const void* base, CUtensorMapDataType type, int rank,
+               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[5];
@@ -93,7 +98,7 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
     estr[i] = 1;
     if (i + 1 < rank) gstr[i] = strides_bytes[i];
   }
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+  CUresult r = fn(map, type, (cuuint32_t)rank, const_cast<void*>(base),
                   gdim, gstr, bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

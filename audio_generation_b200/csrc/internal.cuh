@@ -107,6 +107,16 @@ cudaError_t launch_norm_modulate(const LayoutView& L, int B, int H, int chunk_sh
                                  const float* table, const float* tmod, void* h,
                                  cudaStream_t st);
 
+// The same normalised, modulated rows as e4m3 codes [rows, H] with one scale
+// per row (max |h| / 448), and bf16 weight rows [rows, K] as e4m3 codes with
+// one scale per row.
+cudaError_t launch_norm_modulate_e4m3(const LayoutView& L, int B, int H, int chunk_shift,
+                                      int chunk_scale, float eps, const void* x, bool x_f32,
+                                      const float* table, const float* tmod, void* codes,
+                                      float* row_scale, cudaStream_t st);
+cudaError_t launch_quantize_rows_e4m3(int rows, int K, const void* w, void* codes,
+                                      float* row_scale, cudaStream_t st);
+
 // The prologue's fp32 GEMMs run either on the CUDA cores or, for many distinct
 // timesteps, as bf16 tensor-core GEMMs over three-way bf16 splits of both
 // operands (allow_split = false forces the first form). Workspace bytes for
@@ -142,11 +152,19 @@ struct GemmEpiArgs {
   const float* table = nullptr;
   const float* tmod = nullptr;
   int gate_chunk = 0;
+  // e4m3 GEMMs: per-row activation scales [M] and per-column weight scales [N]
+  const float* a_scale = nullptr;
+  const float* b_scale = nullptr;
 };
 
 // C[M, N] epilogue( A[M, K] . B[N, K]^T ), bf16 in, fp32 accumulate.
 cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void* Bm,
                         const GemmEpiArgs& e, cudaStream_t st);
+
+// The same product on e4m3 codes (A [M, K], B [N, K] bytes) with
+// C[m, n] = a_scale[m] * b_scale[n] * (A . B^T)[m, n]; EPI_QKV or EPI_SWIGLU.
+cudaError_t launch_gemm_e4m3(int epi, int M, int N, int K, const void* A, const void* Bm,
+                             const GemmEpiArgs& e, cudaStream_t st);
 
 cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, const void* k,
                              const void* v, void* o, cudaStream_t st);

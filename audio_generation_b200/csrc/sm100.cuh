@@ -212,6 +212,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor for kind::f8f6f4 with e4m3 A/B (format code 0) and
+// fp32 D: the same fields as kind::f16, with the 8-bit formats.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                        // D format: f32
+         | (0u << 7)                      // A format: e4m3
+         | (0u << 10)                     // B format: e4m3
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
 // Per-warpgroup register budget changes (all four warps of a warpgroup execute
 // these). The budgets after a split must add up to at most the registers the
 // block was launched with, or the increase would wait forever.
@@ -330,6 +340,22 @@ __device__ __forceinline__ void umma_ss_w_pair_elect(uint32_t d_tmem, uint32_t a
       "mov.b64 da, {%1, %2};\n\t"
       "mov.b64 db, {%3, %4};\n\t"
       "@e tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same pair MMA on e4m3 operands (kind::f8f6f4, K = 32 per instruction:
+// the same 32 bytes of a 128-byte swizzled row as K = 16 of bf16).
+__device__ __forceinline__ void umma_ss_w_pair_elect_f8(uint32_t d_tmem, uint32_t a_lo,
+                                                        uint32_t a_hi, uint32_t b_lo,
+                                                        uint32_t b_hi, uint32_t idesc,
+                                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 da, db;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
       "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }

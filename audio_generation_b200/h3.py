@@ -66,6 +66,11 @@ class h3_io_weights(ctypes.Structure):
         "out_table", "w_head_video", "w_head_audio")]
 
 
+class h3_block_weights_e4m3(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_qkv_codes", "w_qkv_scales", "w13_codes", "w13_scales")]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -96,6 +101,11 @@ _SIGNATURES = {
                                   _vp]),
     "h3_block_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _vp,
                               _vp, _vp, _i, _vp, _sz, _vp]),
+    "h3_quantize_e4m3_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "h3_workspace_size_e4m3": (_sz, [ctypes.POINTER(h3_dims), _i, _i]),
+    "h3_block_forward_e4m3": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights),
+                                   ctypes.POINTER(h3_block_weights_e4m3), _vp, _vp, _vp, _i, _vp,
+                                   _sz, _vp]),
     "h3_layout_reduce": (_i, [ctypes.POINTER(h3_dims), _vp, _vp, _vp, ctypes.POINTER(_vp)]),
     "h3_stack_reduced_workspace_size": (_sz, [ctypes.POINTER(h3_dims), _vp, _vp, _i]),
     "h3_stack_forward_reduced": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights),
@@ -379,3 +389,24 @@ def h3_stack_forward_reduced(dims: h3_dims, weights: Sequence[h3_block_weights],
                                           reduced.handle, r0, r1, _ptr(tmod), _ptr(x), B, _ptr(ws),
                                           ws_bytes, _stream(stream)),
            "h3_stack_forward_reduced")
+
+
+def h3_quantize_e4m3_rows(w, rows: int, K: int, codes, scales, stream=None) -> None:
+    _check(lib().h3_quantize_e4m3_rows(_ptr(w), rows, K, _ptr(codes), _ptr(scales),
+                                       _stream(stream)), "h3_quantize_e4m3_rows")
+
+
+def make_block_weights_e4m3(w_qkv_codes, w_qkv_scales, w13_codes, w13_scales):
+    return h3_block_weights_e4m3(*[_ptr(t) for t in (w_qkv_codes, w_qkv_scales, w13_codes,
+                                                     w13_scales)])
+
+
+def h3_workspace_size_e4m3(dims: h3_dims, B: int, S: int) -> int:
+    return lib().h3_workspace_size_e4m3(ctypes.byref(dims), B, S)
+
+
+def h3_block_forward_e4m3(dims: h3_dims, weights: h3_block_weights, w8: h3_block_weights_e4m3,
+                          layout: Layout, tmod, x, B: int, ws, ws_bytes: int, stream=None) -> None:
+    _check(lib().h3_block_forward_e4m3(ctypes.byref(dims), ctypes.byref(weights), ctypes.byref(w8),
+                                       layout.handle, _ptr(tmod), _ptr(x), B, _ptr(ws), ws_bytes,
+                                       _stream(stream)), "h3_block_forward_e4m3")

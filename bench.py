@@ -684,6 +684,85 @@ def run_stack(args):
     return 0
 
 
+def run_e4m3(args):
+    """--e4m3: the block step of the workload with its QKV and W1 || W3 GEMMs on
+    e4m3 operands (h3_block_forward_e4m3; weights quantized once, before timing).
+    Own JSON line; TFLOP/s over the same algorithmic flops as the bf16 block."""
+    import torch
+    from audio_generation_b200 import h3
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    dims = FULL_DIMS
+    d = h3.make_dims(dims)
+    cfg = args.workload
+    L = config_layout(cfg)
+    S, V = L.S, L.n_valid
+    bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(
+        torch.bfloat16)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+    w = block_weights(dims, cfg, 0)
+    wd = {k: bits(getattr(w, k)) for k in ("w_qkv", "q_norm", "k_norm", "w_o", "w13", "w2")}
+    wd["ada_table"] = f32(w.ada_table)
+    cw = h3.make_block_weights(wd["w_qkv"], wd["q_norm"], wd["k_norm"], wd["w_o"], wd["w13"],
+                               wd["w2"], wd["ada_table"])
+    q8 = {}
+    for name in ("w_qkv", "w13"):
+        rows, K = getattr(w, name).shape
+        q8[name] = (torch.empty((rows, K), dtype=torch.uint8, device=device),
+                    torch.empty(rows, dtype=torch.float32, device=device))
+        h3.h3_quantize_e4m3_rows(wd[name], rows, K, q8[name][0], q8[name][1])
+    w8 = h3.make_block_weights_e4m3(q8["w_qkv"][0], q8["w_qkv"][1], q8["w13"][0], q8["w13"][1])
+    layout = h3.h3_layout_prepare(d, S, L.n_t, f32(L.pos), i32(L.tags), i32(L.t_idx),
+                                  i32(L.video_idx), i32(L.audio_idx), i32(L.text_idx))
+    pw = prologue_weights(dims, cfg)
+    tws_b = h3.h3_timestep_workspace_size(d, L.n_t)
+    tws = torch.empty(tws_b, dtype=torch.uint8, device=device)
+    tmod = torch.empty((L.n_t, 6, dims.hidden), dtype=torch.float32, device=device)
+    h3.h3_timestep_modulation(d, L.n_t, f32(L.timestep), f32(pw.w_t1), f32(pw.w_t2),
+                              f32(pw.w_proj), tmod, tws, tws_b)
+    del tws
+    x = bits(activations(dims, cfg, S, 1))
+    ws_b = h3.h3_workspace_size_e4m3(d, 1, S)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        h3.h3_block_forward_e4m3(d, cw, w8, layout, tmod, x, 1, ws, ws_b, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    gpu_id = torch.cuda.get_device_properties(device).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        time.sleep(0.3)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    if h3.h3_layout_error(layout) != h3.H3_OK:
+        raise RuntimeError("device error word set during the e4m3 run")
+    ms = e0.elapsed_time(e1) / args.steps
+    tflops = block_flops(dims, V) / (ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    line = {
+        "metric": METRIC + " [e4m3 QKV and W1||W3 operands]", "value": S / (ms * 1e-3),
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "e4m3 (QKV, W1||W3) + bf16",
+        "data": "synthetic (seeded random-init weights and activations)",
+        "config": {"workload": WORKLOADS[cfg], "S": S, "valid_rows": V},
+        "tflops": tflops, "frac_of_bf16_burst_peak": tflops / peaks["bf16_tflops"],
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    layout.close()
+    return 0
+
+
 FORWARD_WORKLOAD = ("full MiniMax-H3 transformer forward: fp32 patch projections (96 / 32 "
                     "channels), text projection (5120) and 2 refiner blocks, the 50-block stack "
                     "over the 16384-row padded layout (15872 valid rows, two timesteps), norm_out "
@@ -799,6 +878,8 @@ def main(argv=None):
                     help="skip the masked-attention measurement on the padded layout")
     ap.add_argument("--stack", action="store_true",
                     help="time the 50-block stack forward instead (one GPU, own JSON line)")
+    ap.add_argument("--e4m3", action="store_true",
+                    help="time the block with e4m3 QKV and W1||W3 operands instead (own JSON line)")
     ap.add_argument("--forward", action="store_true",
                     help="time the whole transformer forward instead (one GPU, own JSON line)")
     args = ap.parse_args(argv)
@@ -811,6 +892,8 @@ def main(argv=None):
         return run_stack(args)
     if args.forward:
         return run_forward(args)
+    if args.e4m3:
+        return run_e4m3(args)
     return run_gpu(args, world, rank, local)
 
 

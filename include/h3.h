@@ -281,6 +281,43 @@ H3_API h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* w
                            h3_layout_t layout, const float* tmod, void* x, int B, void* ws,
                            size_t ws_bytes, h3_stream_t stream);
 
+/* ---- 8-bit (e4m3) inputs for the QKV and W1 || W3 GEMMs ---- */
+
+/* "MiniMax H3 Inference Engine voor Mac computers", sections "Profiling en
+ * diagnostische pads" and "Sampler en DiT controls": an 8-bit MLP and 8-bit QKV
+ * projections with one activation scale per row. Here (reading): e4m3 codes
+ * for both operands of the QKV and W1 || W3 GEMMs (tcgen05 kind::f8f6f4), one
+ * scale per activation row (its largest |h| / 448, computed by the norm kernel)
+ * and one per weight row; the product of the scales is applied to the fp32 dot
+ * product of the codes. The O and W2 GEMMs and everything else stay as in
+ * h3_block_forward. */
+
+/* Weight rows [rows, K] bf16 -> e4m3 codes [rows, K] (one byte each) and
+ * scales [rows] f32: scale = max|w| / 448 (1 for an all-zero row), code =
+ * e4m3(w / scale), round to nearest even, saturating. K % 16 == 0. Enqueues. */
+H3_API h3_status h3_quantize_e4m3_rows(const void* w, int rows, int K, void* codes, float* scales,
+                                       h3_stream_t stream);
+
+/* The 8-bit operands of one block (DEVICE pointers, from h3_quantize_e4m3_rows
+ * applied to the block's w_qkv [3*NH*D, H] and w13 [2F, H]). */
+typedef struct {
+  const void* w_qkv_codes;
+  const float* w_qkv_scales;
+  const void* w13_codes;
+  const float* w13_scales;
+} h3_block_weights_e4m3;
+
+/* Workspace bytes of h3_block_forward_e4m3: h3_workspace_size plus the codes
+ * [B*S, H] and scales [B*S] of the activation rows. */
+H3_API size_t h3_workspace_size_e4m3(const h3_dims* dims, int B, int S);
+
+/* h3_block_forward with the QKV and W1 || W3 GEMMs on e4m3 operands (the bf16
+ * w_qkv and w13 of `weights` are not read). hidden % 128 == 0. */
+H3_API h3_status h3_block_forward_e4m3(const h3_dims* dims, const h3_block_weights* weights,
+                                       const h3_block_weights_e4m3* w8, h3_layout_t layout,
+                                       const float* tmod, void* x, int B, void* ws,
+                                       size_t ws_bytes, h3_stream_t stream);
+
 /* ---- token reduction in the middle blocks ---- */
 
 /* Build the token-reduced layout of `full` ("MiniMax H3 Inference Engine voor

@@ -474,6 +474,98 @@ def denoiser_forward(video: np.ndarray, audio: np.ndarray, text: np.ndarray, dw,
 
 
 # --------------------------------------------------------------------------
+# 8-bit GEMM inputs for the QKV and W1 || W3 projections  [ME: "Profiling en
+# diagnostische pads" and "Sampler en DiT controls": an 8-bit MLP and 8-bit QKV
+# projections, with one activation scale per row]
+#
+# Reading (B200 form): the e4m3 format (1 sign, 4 exponent bits of bias 7, 3
+# mantissa bits, largest finite value 448, no infinities) for both operands;
+# one scale per activation row (that row's largest |h| / 448) and one per
+# weight row (output channel); the product of the two scales is applied to the
+# fp32 dot product of the codes. The scale and the division are float32, as on
+# the device, so that both sides round the same values to the same codes.
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Nearest e4m3 value (ties to even), saturating at +-448: normal numbers
+    2^(e-7) (1 + m/8), e = 1..15 (e = 15 only up to m = 6), subnormals
+    2^-6 m/8; the grid spacing of a value in [2^k, 2^(k+1)) is 2^(k-3), below
+    2^-6 it is 2^-9."""
+    a = np.abs(np.asarray(x, F))
+    k = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
+    step = 2.0 ** (np.maximum(k, -6.0) - 3.0)
+    q = a / step
+    r = np.floor(q)
+    frac = q - r
+    up = (frac > 0.5) | ((frac == 0.5) & (np.mod(r, 2) == 1))
+    v = (r + up) * step
+    v = np.minimum(v, E4M3_MAX)
+    return np.where(np.asarray(x, F) < 0, -v, v)
+
+
+def row_scales_f32(a: np.ndarray) -> np.ndarray:
+    """Per-row scale max|a| / 448 in float32 (1 for an all-zero row)."""
+    m = np.max(np.abs(np.asarray(a, np.float32)), axis=-1)
+    s = (m / np.float32(E4M3_MAX)).astype(np.float32)
+    return np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+
+
+def quantize_rows_e4m3(a: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """(codes as their e4m3 values, float32 row scales): a ~= codes * scale."""
+    a32 = np.asarray(a, np.float32)
+    s = row_scales_f32(a32)
+    return e4m3_round((a32 / s[:, None]).astype(np.float32)), s
+
+
+def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    return np.asarray(codes, F) * np.asarray(scales, F)[:, None]
+
+
+def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims) -> np.ndarray:
+    """The block with its QKV and W1 || W3 GEMMs on e4m3 inputs: the norm outputs
+    h and h2 quantized per row (their values held in float32, as the device
+    holds them) and the bf16 weights per output channel; everything else as in
+    block_forward. (B = 1 or more; padding rows unchanged.)"""
+    import copy
+    wq = copy.copy(w)
+    for name in ("w_qkv", "w13"):
+        wf = bf16_to_f64(getattr(w, name)).astype(np.float32)
+        codes, sc = quantize_rows_e4m3(wf)
+        setattr(wq, name, dequantize_rows(codes, sc))
+    x = np.asarray(x, F)
+    tags = np.asarray(layout.tags)
+    if tags.shape[0] == 0:
+        return x.copy()
+    pad = tags < 0
+    m = row_modulation(tags, layout.t_idx, w.ada_table, tmod)
+    out = np.empty_like(x)
+    NH, D = dims.heads, dims.head_dim
+    inv = rope_inv_freq(dims.rope_freq_dim, dims.rope_theta)
+    for b in range(x.shape[0]):
+        h = norm_modulate(x[b], m[:, 0], m[:, 1], dims.norm_eps)
+        hq = dequantize_rows(*quantize_rows_e4m3(h))
+        wqs, wks, wvs = split_qkv_weight(wq.w_qkv, NH, D)
+        n = h.shape[0]
+        q = rope_apply(rms_norm((hq @ wqs.T).reshape(n, NH, D), bf16_to_f64(w.q_norm),
+                                dims.qk_norm_eps), layout.pos, inv)
+        k = rope_apply(rms_norm((hq @ wks.T).reshape(n, NH, D), bf16_to_f64(w.k_norm),
+                                dims.qk_norm_eps), layout.pos, inv)
+        v = (hq @ wvs.T).reshape(n, NH, D)
+        o = attention(q, pad, k, v, pad)
+        x1 = out_project_residual(x[b], o, m[:, 2], w.w_o)
+        h2 = norm_modulate(x1, m[:, 3], m[:, 4], dims.norm_eps)
+        h2q = dequantize_rows(*quantize_rows_e4m3(h2))
+        w1, w3 = split_w13(wq.w13, dims.ffn)
+        g = silu(h2q @ w1.T) * (h2q @ w3.T)
+        y = ffn_down_residual(x1, g, m[:, 5], w.w2)
+        out[b] = np.where(pad[:, None], x[b], y)
+    return out
+
+
+# --------------------------------------------------------------------------
 # Token reduction in the middle blocks  [ME: "Token-reduction internals": after
 # block 3 adjacent horizontal target-video tokens are paired, text, audio and
 # reference tokens stay exact; the full-resolution state is kept as a bypass

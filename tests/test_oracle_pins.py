@@ -1015,3 +1015,50 @@ def test_core_reuse_with_the_same_latents_is_the_full_forward():
     xr = v2 @ np.asarray(dw.w_patch_video).T + res[L.video_idx]
     np.testing.assert_allclose(rv2, O.output_head(xr, m[:, 0], m[:, 1], dw.w_head_video, 1e-5),
                                rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- 8-bit GEMM inputs
+
+def test_e4m3_rounding_matches_torch_and_the_format():
+    """In-range values against torch's float8_e4m3fn conversion (round to
+    nearest even), plus the format's landmarks by hand: 448 the largest finite
+    value, 2^-9 the smallest subnormal, steps of 2^(k-3) in [2^k, 2^(k+1))."""
+    g = np.random.default_rng(8)
+    x = np.concatenate([g.standard_normal(20000) * 50, g.uniform(-448, 448, 20000),
+                        g.standard_normal(5000) * 0.01, np.linspace(-3, 3, 4001)])
+    ref = torch.tensor(x, dtype=torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.e4m3_round(x.astype(np.float32)), ref)
+    assert O.e4m3_round(np.array([500.0, -1e6]))[0] == 448.0
+    assert O.e4m3_round(np.array([-1e6]))[0] == -448.0
+    np.testing.assert_array_equal(O.e4m3_round(np.array([2.0 ** -9, 2.0 ** -10, 1.5 * 2.0 ** -10])),
+                                  [2.0 ** -9, 0.0, 2.0 ** -9])
+    # 1.0625 is halfway between 1 and 1.125: ties to the even code (1.0)
+    np.testing.assert_array_equal(O.e4m3_round(np.array([1.0625, 1.1875, 17.0, 19.0])),
+                                  [1.0, 1.25, 16.0, 20.0])
+
+
+def test_row_quantization_round_trip():
+    g = np.random.default_rng(9)
+    a = (g.standard_normal((7, 300)) * np.array([1e-3, 1, 30, 0, 5, 1e4, 2])[:, None])
+    codes, s = O.quantize_rows_e4m3(a)
+    assert s.dtype == np.float32 and s[3] == 1.0 and np.all(codes[3] == 0)
+    assert np.all(np.abs(codes) <= 448) and np.all(np.max(np.abs(codes), 1)[[0, 1, 2, 4, 5, 6]] == 448)
+    back = O.dequantize_rows(codes, s)
+    ok = np.abs(a) > 2.0 ** -6 * s[:, None]  # normal range: relative error <= 2^-4
+    assert np.all(np.abs(back - a)[ok] <= 2.0 ** -4 * np.abs(a)[ok] * (1 + 1e-6))
+
+
+def test_fp8_block_is_close_to_the_block_and_keeps_padding():
+    """The 8-bit block moves x like the block, within the quantization error
+    (a few % of the update), and leaves padding rows unchanged."""
+    L = random_layout(64, 3, pad_runs=2, max_run=9)
+    w = _weights_big_gates(SMALL, 12)
+    tmod = _tmod_random(L.n_t, SMALL.hidden, 4)
+    x = np.random.default_rng(5).standard_normal((1, L.S, SMALL.hidden))
+    y = O.block_forward(x, w, L, tmod, SMALL)
+    y8 = O.block_forward_fp8(x, w, L, tmod, SMALL)
+    pad = L.tags < 0
+    np.testing.assert_array_equal(y8[0, pad], x[0, pad])
+    d, d8 = y[0, ~pad] - x[0, ~pad], y8[0, ~pad] - x[0, ~pad]
+    r = _rel(d8, d)
+    assert 1e-3 < r < 0.08, r
