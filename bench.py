@@ -545,15 +545,13 @@ def run_gpu(args, world, rank, local):
     return 0
 
 
-def masked_attention(h3, d, dims, device, stream, peaks, reps=10):
-    """The attention kernel alone on the padded 16384-row layout (512 padding
-    rows in four runs; two runs straddle a 128-row tile, so two tiles need the
-    per-key mask and two are skipped whole). Q, K and V are seeded N(0, 1) bf16
-    rows, the scale of q and k after the per-head RMSNorm. Reports the kernel's
-    mean time and TFLOP/s over the valid work, 4 NH D V^2 for the V valid rows
-    (the padding document is not counted)."""
+def attention_only(h3, d, dims, device, stream, peaks, cfg, reps, warmup=3):
+    """The attention kernel alone on one workload's layout (Q, K, V seeded
+    N(0, 1) bf16, the scale of q and k after the per-head RMSNorm); only the
+    layout tables, q, k, v and o are on the device. Mean time and TFLOP/s over
+    the valid work, 4 NH D V^2 (the padding document is not counted)."""
     import torch
-    L = config_layout(MASKED_CFG)
+    L = config_layout(cfg)
     S, V = L.S, L.n_valid
     to_i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
     pos = torch.from_numpy(np.ascontiguousarray(L.pos, dtype=np.float32)).to(device)
@@ -565,7 +563,7 @@ def masked_attention(h3, d, dims, device, stream, peaks, reps=10):
     q, k, v = (torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(
         torch.bfloat16) for _ in range(3))
     o = torch.empty((1, S, dims.attn_width), dtype=torch.bfloat16, device=device)
-    for _ in range(3):
+    for _ in range(warmup):
         h3.h3_attention(d, layout, 1, q, k, v, o, stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(device)
@@ -575,14 +573,39 @@ def masked_attention(h3, d, dims, device, stream, peaks, reps=10):
     e1.record(stream)
     torch.cuda.synchronize(device)
     if h3.h3_layout_error(layout) != h3.H3_OK:
-        raise RuntimeError("device error word set during the masked attention run")
+        raise RuntimeError("device error word set during the attention run")
     layout.close()
     ms = e0.elapsed_time(e1) / reps
     tf = 4.0 * dims.heads * dims.head_dim * float(V) ** 2 / (ms * 1e-3) / 1e12
-    return {"workload": WORKLOADS[MASKED_CFG], "S": S, "valid_rows": V, "launches": reps,
-            "ms": round(ms, 4), "tflops_valid": round(tf, 1),
+    return {"workload": WORKLOADS.get(cfg, CONFIG_NAMES_SHORT.get(cfg)), "S": S,
+            "valid_rows": V, "launches": reps, "ms": round(ms, 4), "tflops_valid": round(tf, 1),
             "frac_of_peak": round(tf / peaks["bf16_tflops"], 3), "peak_kind": "burst",
             "frac_of_sustained_peak": round(tf / peaks["bf16_tflops_sustained"], 3)}
+
+
+CONFIG_NAMES_SHORT = {5: "the 16384-row padded layout of the 50-block stack"}
+
+
+def run_attention_only(args):
+    """--attention-only: the attention kernel alone on the workload's layout
+    (own JSON line); with little on the device, for profiler captures."""
+    import torch
+    from audio_generation_b200 import h3
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    dims = FULL_DIMS
+    res = attention_only(h3, h3.make_dims(dims), dims, device, torch.cuda.current_stream(device),
+                         load_peaks(), args.workload, args.steps, args.warmup)
+    print(json.dumps(dict(res, metric="attention TFLOP/s over the valid work (bf16, 1xB200)",
+                          unit="TFLOP/s", value=res["tflops_valid"])))
+    return 0
+
+
+def masked_attention(h3, d, dims, device, stream, peaks, reps=10):
+    """The attention kernel alone on the padded 16384-row layout (512 padding
+    rows in four runs; two runs straddle a 128-row tile, so two tiles need the
+    per-key mask and two are skipped whole), through attention_only."""
+    return attention_only(h3, d, dims, device, stream, peaks, MASKED_CFG, reps)
 
 
 STACK_CFG = 5
@@ -878,6 +901,8 @@ def main(argv=None):
                     help="skip the masked-attention measurement on the padded layout")
     ap.add_argument("--stack", action="store_true",
                     help="time the 50-block stack forward instead (one GPU, own JSON line)")
+    ap.add_argument("--attention-only", action="store_true",
+                    help="time the attention kernel alone on the workload (own JSON line)")
     ap.add_argument("--e4m3", action="store_true",
                     help="time the block with e4m3 QKV and W1||W3 operands instead (own JSON line)")
     ap.add_argument("--forward", action="store_true",
@@ -894,6 +919,8 @@ def main(argv=None):
         return run_forward(args)
     if args.e4m3:
         return run_e4m3(args)
+    if args.attention_only:
+        return run_attention_only(args)
     return run_gpu(args, world, rank, local)
 
 
