@@ -428,7 +428,10 @@ h3_status h3_qkv_rope(const h3_dims* dims, h3_layout_t L, int B, const void* h, 
 
 h3_status h3_attention(const h3_dims* dims, h3_layout_t L, int B, const void* q, const void* k,
                        const void* v, void* o, h3_stream_t stream) {
-  H3_TRY(check_dims(dims));
+  // Attention alone needs only head_dim 128 and any head count (a rank of the
+  // sequence-parallel block runs it on heads / P heads).
+  if (!dims) return H3_ERR_ARG;
+  if (dims->head_dim != 128 || dims->heads <= 0 || dims->heads > 65535) return H3_ERR_SHAPE;
   if (!L || B < 0 || !q || !k || !v || !o) return H3_ERR_ARG;
   H3_TRY(check_batch(L, B));
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return H3_ERR_ALIGN;

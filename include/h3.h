@@ -240,7 +240,8 @@ H3_API h3_status h3_qkv_rope(const h3_dims* dims, h3_layout_t layout, int B, con
  * result: rows of 128-row tiles that hold only padding are written as zeros;
  * padding rows inside mixed tiles hold finite values that every later step
  * ignores (they are never read back into x). q, k, v [B, NH, S, D] bf16 ->
- * o [B, S, NH*D] bf16. */
+ * o [B, S, NH*D] bf16. Only head_dim (128) and heads (any count >= 1) of dims
+ * are used here, so a caller may run it on a subset of the heads. */
 H3_API h3_status h3_attention(const h3_dims* dims, h3_layout_t layout, int B, const void* q,
                        const void* k, const void* v, void* o, h3_stream_t stream);
 

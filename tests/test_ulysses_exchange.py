@@ -1,0 +1,60 @@
+"""The head <-> sequence exchange of the sequence-parallel block between real
+processes (gloo, world size 2 and 4, CPU tensors): after seq_to_heads every
+rank holds every row of its heads in packed order; heads_to_seq gives each rank
+its rows of every head, in head order; the two are inverse to each other."""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from audio_generation_b200.ulysses import heads_to_seq, seq_to_heads
+
+
+def _port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        NH, S, D = 4 * world, 6 * world, 3
+        full = torch.arange(NH * S * D, dtype=torch.float32).view(NH, S, D)  # [heads, rows, D]
+        Sr, NHl = S // world, NH // world
+        mine = full[:, rank * Sr:(rank + 1) * Sr].clone()
+        a2a = lambda out, inp: dist.all_to_all_single(out, inp)
+        got = seq_to_heads(mine, world, a2a)
+        ok1 = torch.equal(got, full[rank * NHl:(rank + 1) * NHl])
+        # o [S, NHl * D] of this rank's heads -> this rank's rows of every head
+        o_heads = full[rank * NHl:(rank + 1) * NHl].permute(1, 0, 2).reshape(S, NHl * D)
+        back = heads_to_seq(o_heads, world, a2a)
+        want = full[:, rank * Sr:(rank + 1) * Sr].permute(1, 0, 2).reshape(Sr, NH * D)
+        ok2 = torch.equal(back, want)
+        q.put((rank, bool(ok1), bool(ok2)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_exchange_between_processes(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    assert res == [(r, True, True) for r in range(world)]
