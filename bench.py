@@ -534,6 +534,15 @@ def run_gpu(args, world, rank, local):
         "gpu_launches": len(launches) * args.steps,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_stack:
+        # the 50-block stack over the padded 16384-row layout, two timed forwards
+        del x_host, out_host, xd, ws
+        torch.cuda.empty_cache()
+        st = stack_measure(2, 1)
+        line["stack_config5"] = {k: st[k] for k in ("value", "unit", "ms_per_step", "tflops",
+                                                    "frac_of_sustained_peak", "frac_of_burst_peak",
+                                                    "clocks", "steps", "warmup")}
+        line["stack_config5"]["workload"] = st["config"]["workload"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_baseline(cfg, args.ref_rows, 3)
     if rank == 0:
@@ -616,11 +625,17 @@ STACK_WORKLOAD = ("full-width MiniMax-H3 50-block stack forward, S=16384 packed 
 
 
 def run_stack(args):
-    """--stack: the 50-block stack forward on one GPU (layout prepared once, the
+    """--stack: the 50-block stack forward on one GPU, one JSON line."""
+    print(json.dumps(stack_measure(args.steps, args.warmup)))
+    return 0
+
+
+def stack_measure(steps, warmup):
+    """The 50-block stack forward on one GPU (layout prepared once, the
     per-forward prologue for the two timesteps, then the stack with the valid rows
-    gathered into an fp32 stream and scattered back). Prints one JSON line with
-    the forward time, valid rows/s and TFLOP/s (algorithmic flops of 50 blocks
-    over the valid rows and the valid document)."""
+    gathered into an fp32 stream and scattered back): forward time, valid rows/s
+    and TFLOP/s (algorithmic flops of 50 blocks over the valid rows and the valid
+    document)."""
     import torch
     from audio_generation_b200 import h3
 
@@ -672,7 +687,7 @@ def run_stack(args):
         h3.h3_timestep_modulation(d, L.n_t, t_dev, w1, w2p, wp, tmod, tws, tws_b, stream)
         h3.h3_stack_forward(d, cws, layout, tmod, x, 1, ws, ws_b, stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         forward()
     torch.cuda.synchronize(device)
     gpu_id = torch.cuda.get_device_properties(device).uuid
@@ -681,30 +696,29 @@ def run_stack(args):
     with ClockSampler(gpu_id) as clk:
         time.sleep(0.3)
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             forward()
         e1.record(stream)
         torch.cuda.synchronize(device)
     if h3.h3_layout_error(layout) != h3.H3_OK:
         raise RuntimeError("device error word set during the stack run")
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = e0.elapsed_time(e1) / steps
     flops = STACK_BLOCKS * block_flops(dims, V)
     peaks = load_peaks()
     tflops = flops / (ms * 1e-3) / 1e12
     line = {
         "metric": "valid packed rows/s per 50-block stack forward (bf16, 1xB200)",
-        "value": V / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16",
+        "value": V / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16",
         "data": "synthetic (seeded random-init weights and activations)",
         "config": {"workload": STACK_WORKLOAD, "S": S, "valid_rows": V, "blocks": STACK_BLOCKS,
                    "n_t": int(L.n_t)},
         "tflops": tflops, "frac_of_sustained_peak": tflops / peaks["bf16_tflops_sustained"],
         "frac_of_burst_peak": tflops / peaks["bf16_tflops"], "clocks": clk.summary(),
-        "gpu_launches": args.steps * (4 + 2 + 7 * STACK_BLOCKS),  # prologue, gather / scatter, blocks
+        "gpu_launches": steps * (4 + 2 + 7 * STACK_BLOCKS),  # prologue, gather / scatter, blocks
     }
-    print(json.dumps(line))
     layout.close()
-    return 0
+    return line
 
 
 def run_e4m3(args):
@@ -897,6 +911,8 @@ def main(argv=None):
     ap.add_argument("--ref-rows", type=int, default=256,
                     help="query rows per bounded oracle sample (one reference step)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stack", action="store_true",
+                    help="skip the 50-block stack measurement added to the block line")
     ap.add_argument("--no-masked", action="store_true",
                     help="skip the masked-attention measurement on the padded layout")
     ap.add_argument("--stack", action="store_true",
