@@ -524,11 +524,18 @@ def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return np.asarray(codes, F) * np.asarray(scales, F)[:, None]
 
 
-def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims) -> np.ndarray:
+def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
+                      emulate: bool = False) -> np.ndarray:
     """The block with its QKV and W1 || W3 GEMMs on e4m3 inputs: the norm outputs
     h and h2 quantized per row (their values held in float32, as the device
     holds them) and the bf16 weights per output channel; everything else as in
-    block_forward. (B = 1 or more; padding rows unchanged.)"""
+    block_forward. (B = 1 or more; padding rows unchanged.)
+
+    ``emulate`` rounds to bf16 where the device stores bf16 in this block (q, k, v
+    after RoPE, P, o, x1, g, x2; h and h2 go from fp32 straight to codes). A
+    code is an integer that floating point decides: compared with the device,
+    the reference must take that decision from the values the device holds, so
+    the norm2 input x1 has to be the bf16 value the device stored."""
     import copy
     wq = copy.copy(w)
     for name in ("w_qkv", "w13"):
@@ -549,18 +556,18 @@ def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims) -> np.nd
         hq = dequantize_rows(*quantize_rows_e4m3(h))
         wqs, wks, wvs = split_qkv_weight(wq.w_qkv, NH, D)
         n = h.shape[0]
-        q = rope_apply(rms_norm((hq @ wqs.T).reshape(n, NH, D), bf16_to_f64(w.q_norm),
-                                dims.qk_norm_eps), layout.pos, inv)
-        k = rope_apply(rms_norm((hq @ wks.T).reshape(n, NH, D), bf16_to_f64(w.k_norm),
-                                dims.qk_norm_eps), layout.pos, inv)
-        v = (hq @ wvs.T).reshape(n, NH, D)
-        o = attention(q, pad, k, v, pad)
-        x1 = out_project_residual(x[b], o, m[:, 2], w.w_o)
+        q = _store(rope_apply(rms_norm((hq @ wqs.T).reshape(n, NH, D), bf16_to_f64(w.q_norm),
+                                       dims.qk_norm_eps), layout.pos, inv), emulate)
+        k = _store(rope_apply(rms_norm((hq @ wks.T).reshape(n, NH, D), bf16_to_f64(w.k_norm),
+                                       dims.qk_norm_eps), layout.pos, inv), emulate)
+        v = _store((hq @ wvs.T).reshape(n, NH, D), emulate)
+        o = attention(q, pad, k, v, pad, emulate)
+        x1 = out_project_residual(x[b], o, m[:, 2], w.w_o, emulate)
         h2 = norm_modulate(x1, m[:, 3], m[:, 4], dims.norm_eps)
         h2q = dequantize_rows(*quantize_rows_e4m3(h2))
         w1, w3 = split_w13(wq.w13, dims.ffn)
-        g = silu(h2q @ w1.T) * (h2q @ w3.T)
-        y = ffn_down_residual(x1, g, m[:, 5], w.w2)
+        g = _store(silu(h2q @ w1.T) * (h2q @ w3.T), emulate)
+        y = ffn_down_residual(x1, g, m[:, 5], w.w2, emulate)
         out[b] = np.where(pad[:, None], x[b], y)
     return out
 

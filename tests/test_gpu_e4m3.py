@@ -6,6 +6,14 @@ projections, one activation scale per row). The oracle quantizes at the same
 points (oracle.h3_oracle.block_forward_fp8), so the GPU block is held to the
 same tolerance as the bf16 block against it; the weight codes and scales, whose
 inputs are exact on both sides, are compared bit for bit.
+
+An e4m3 code is an integer decided by floating point, and one code step is 6-12 %
+of a value: the reference must decide the codes of h2 from the norm2 input the
+device holds, x1 stored in bf16. The oracle's 8-bit block is therefore compared
+in its bf16-storage emulation (bf16 where the device stores bf16; h and h2 go
+from fp32 straight to codes on both sides). Against the float64 reference
+without that emulation the norm2 input differs by bf16 rounding, which moves a
+few % of the h2 codes by one step: ~1-2 % differences in x_out.
 """
 
 import numpy as np
@@ -74,9 +82,10 @@ def test_e4m3_block_tiny_workload():
     got = gpu_block_e4m3(dims, L, w, gpu_tmod(dims, L.timestep, pw), xb, 1)[0]
     x0 = O.bf16_to_f64(xb[0])
     tm = O.timestep_modulation(L.timestep, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim, dims.hidden)
-    ref = O.block_forward_fp8(x0[None], w, L, tm, dims)[0]
+    ref = O.block_forward_fp8(x0[None], w, L, tm, dims, emulate=True)[0]
     pad = L.tags < 0
     assert_close(got, ref, what="e4m3 block x_out")
+    assert rel_l2(got[~pad] - x0[~pad], ref[~pad] - x0[~pad]) < 0.1
     np.testing.assert_array_equal(got[pad], x0[pad])
 
 
@@ -93,14 +102,14 @@ def test_e4m3_block_small_amplified(S, seed):
     pad = L.tags < 0
     for b in range(B):
         x0 = O.bf16_to_f64(xb[b])
-        ref = O.block_forward_fp8(x0[None], w, L, tm, dims)[0]
+        ref = O.block_forward_fp8(x0[None], w, L, tm, dims, emulate=True)[0]
         assert_close(got[b], ref, what=f"e4m3 x_out b={b}", storage_rounding=True)
         assert_close(got[b, ~pad] - x0[~pad], ref[~pad] - x0[~pad], what="e4m3 update",
                      mabs=np.inf)
         np.testing.assert_array_equal(got[b, pad], x0[pad])
         # the 8-bit block is near the bf16 block: a few % of the update
         full = O.block_forward(x0[None], w, L, tm, dims)[0]
-        assert rel_l2(ref[~pad] - x0[~pad], full[~pad] - x0[~pad]) < 0.1
+        assert rel_l2(got[b, ~pad] - x0[~pad], full[~pad] - x0[~pad]) < 0.1
 
 
 def test_e4m3_block_full_width():
@@ -114,7 +123,9 @@ def test_e4m3_block_full_width():
     got = gpu_block_e4m3(dims, L, w, gpu_tmod(dims, L.timestep, pw), xb, 1)[0]
     x0 = O.bf16_to_f64(xb[0])
     tm = O.timestep_modulation(L.timestep, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim, dims.hidden)
-    ref = O.block_forward_fp8(x0[None], w, L, tm, dims)[0]
+    ref = O.block_forward_fp8(x0[None], w, L, tm, dims, emulate=True)[0]
     pad = L.tags < 0
     assert_close(got, ref, what="full-width e4m3 x_out")
+    assert_close(got[~pad] - x0[~pad], ref[~pad] - x0[~pad], what="full-width e4m3 update",
+                 mabs=np.inf)
     np.testing.assert_array_equal(got[pad], x0[pad])
