@@ -802,6 +802,74 @@ h3_status h3_quantize_e4m3_rows(const void* w, int rows, int K, void* codes, flo
   return H3_OK;
 }
 
+h3_status h3_norm_modulate_e4m3(const h3_dims* dims, h3_layout_t L, int B, int which,
+                                const void* x, const float* ada_table, const float* tmod,
+                                void* codes, float* scales, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || (which != 0 && which != 1) || !x || !ada_table || !tmod || !codes ||
+      !scales)
+    return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
+  if (!aligned16(x) || !aligned16(ada_table) || !aligned16(tmod) || !aligned16(codes) ||
+      !aligned16(scales))
+    return H3_ERR_ALIGN;
+  const int c0 = which == 0 ? 0 : 3;
+  H3_CUDA(launch_norm_modulate_e4m3(L->view(), B, dims->hidden, c0, c0 + 1, dims->norm_eps, x,
+                                    false, ada_table, tmod, codes, scales, as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_qkv_rope_e4m3(const h3_dims* dims, h3_layout_t L, int B, const void* h_codes,
+                           const float* h_scales, const void* w_codes, const float* w_scales,
+                           const void* q_norm, const void* k_norm, void* q, void* k, void* v,
+                           h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !h_codes || !h_scales || !w_codes || !w_scales || !q_norm || !k_norm ||
+      !q || !k || !v)
+    return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
+  if (!aligned16(h_codes) || !aligned16(h_scales) || !aligned16(w_codes) ||
+      !aligned16(w_scales) || !aligned16(q_norm) || !aligned16(k_norm) || !aligned16(q) ||
+      !aligned16(k) || !aligned16(v))
+    return H3_ERR_ALIGN;
+  if (dims->hidden % 128 != 0) return H3_ERR_SHAPE;
+  GemmEpiArgs e;
+  e.L = L->view();
+  e.B = B;
+  e.NH = dims->heads;
+  e.q = q;
+  e.k = k;
+  e.v = v;
+  e.q_norm = q_norm;
+  e.k_norm = k_norm;
+  e.qk_eps = dims->qk_norm_eps;
+  e.a_scale = h_scales;
+  e.b_scale = w_scales;
+  H3_CUDA(launch_gemm_e4m3(EPI_QKV, B * L->S, 3 * dims->heads * dims->head_dim, dims->hidden,
+                           h_codes, w_codes, e, as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_ffn_up_e4m3(const h3_dims* dims, h3_layout_t L, int B, const void* h2_codes,
+                         const float* h2_scales, const void* w_codes, const float* w_scales,
+                         void* g, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !h2_codes || !h2_scales || !w_codes || !w_scales || !g) return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
+  if (!aligned16(h2_codes) || !aligned16(h2_scales) || !aligned16(w_codes) ||
+      !aligned16(w_scales) || !aligned16(g))
+    return H3_ERR_ALIGN;
+  if (dims->hidden % 128 != 0) return H3_ERR_SHAPE;
+  GemmEpiArgs sg;
+  sg.L = L->view();
+  sg.out = g;
+  sg.a_scale = h2_scales;
+  sg.b_scale = w_scales;
+  H3_CUDA(launch_gemm_e4m3(EPI_SWIGLU, B * L->S, 2 * dims->ffn, dims->hidden, h2_codes, w_codes,
+                           sg, as_stream(stream)));
+  return H3_OK;
+}
+
 size_t h3_workspace_size_e4m3(const h3_dims* dims, int B, int S) {
   if (check_dims(dims) != H3_OK || B < 0 || S < 0) return 0;
   const size_t rows = (size_t)B * S;

@@ -102,6 +102,11 @@ _SIGNATURES = {
     "h3_block_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _vp,
                               _vp, _vp, _i, _vp, _sz, _vp]),
     "h3_quantize_e4m3_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "h3_norm_modulate_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _i, _vp, _vp, _vp, _vp,
+                                   _vp, _vp]),
+    "h3_qkv_rope_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp,
+                              _vp, _vp, _vp, _vp]),
+    "h3_ffn_up_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "h3_workspace_size_e4m3": (_sz, [ctypes.POINTER(h3_dims), _i, _i]),
     "h3_block_forward_e4m3": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights),
                                    ctypes.POINTER(h3_block_weights_e4m3), _vp, _vp, _vp, _i, _vp,
@@ -394,6 +399,28 @@ def h3_stack_forward_reduced(dims: h3_dims, weights: Sequence[h3_block_weights],
 def h3_quantize_e4m3_rows(w, rows: int, K: int, codes, scales, stream=None) -> None:
     _check(lib().h3_quantize_e4m3_rows(_ptr(w), rows, K, _ptr(codes), _ptr(scales),
                                        _stream(stream)), "h3_quantize_e4m3_rows")
+
+
+def h3_norm_modulate_e4m3(dims: h3_dims, layout: Layout, B: int, which: int, x, ada_table, tmod,
+                          codes, scales, stream=None) -> None:
+    _check(lib().h3_norm_modulate_e4m3(ctypes.byref(dims), layout.handle, B, which, _ptr(x),
+                                       _ptr(ada_table), _ptr(tmod), _ptr(codes), _ptr(scales),
+                                       _stream(stream)), "h3_norm_modulate_e4m3")
+
+
+def h3_qkv_rope_e4m3(dims: h3_dims, layout: Layout, B: int, h_codes, h_scales, w_codes,
+                     w_scales, q_norm, k_norm, q, k, v, stream=None) -> None:
+    _check(lib().h3_qkv_rope_e4m3(ctypes.byref(dims), layout.handle, B, _ptr(h_codes),
+                                  _ptr(h_scales), _ptr(w_codes), _ptr(w_scales), _ptr(q_norm),
+                                  _ptr(k_norm), _ptr(q), _ptr(k), _ptr(v), _stream(stream)),
+           "h3_qkv_rope_e4m3")
+
+
+def h3_ffn_up_e4m3(dims: h3_dims, layout: Layout, B: int, h2_codes, h2_scales, w_codes, w_scales,
+                   g, stream=None) -> None:
+    _check(lib().h3_ffn_up_e4m3(ctypes.byref(dims), layout.handle, B, _ptr(h2_codes),
+                                _ptr(h2_scales), _ptr(w_codes), _ptr(w_scales), _ptr(g),
+                                _stream(stream)), "h3_ffn_up_e4m3")
 
 
 def make_block_weights_e4m3(w_qkv_codes, w_qkv_scales, w13_codes, w13_scales):

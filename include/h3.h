@@ -308,6 +308,33 @@ typedef struct {
   const float* w13_scales;
 } h3_block_weights_e4m3;
 
+/* The steps of the 8-bit block, each as in the bf16 step of the same name.
+ * Activation codes are [B*S, H] bytes (row-major, one row per packed row of
+ * each batch element) with scales [B*S] f32: a row's values are code * scale.
+ * All pointers DEVICE, 16-byte aligned; hidden % 128 == 0 for the GEMM steps.
+ *
+ * h3_norm_modulate_e4m3: h3_norm_modulate followed by the per-row quantization
+ * (scale = max|h| / 448 over the row's fp32 h, 1 for an all-zero row; code =
+ * e4m3(h / scale), round to nearest even, saturating). Padding rows get codes 0
+ * and scale 1. */
+H3_API h3_status h3_norm_modulate_e4m3(const h3_dims* dims, h3_layout_t layout, int B, int which,
+                                       const void* x, const float* ada_table, const float* tmod,
+                                       void* codes, float* scales, h3_stream_t stream);
+
+/* h3_qkv_rope on 8-bit operands: the fp32 dot products of h_codes [B*S, H] and
+ * w_codes [3*NH*D, H] (per-row weight scales w_scales [3*NH*D]), times
+ * h_scales[row] * w_scales[col], then QK-norm + RoPE as in h3_qkv_rope. */
+H3_API h3_status h3_qkv_rope_e4m3(const h3_dims* dims, h3_layout_t layout, int B,
+                                  const void* h_codes, const float* h_scales, const void* w_codes,
+                                  const float* w_scales, const void* q_norm, const void* k_norm,
+                                  void* q, void* k, void* v, h3_stream_t stream);
+
+/* h3_ffn_up on 8-bit operands: h2_codes [B*S, H] (scales [B*S]) against the
+ * W1 || W3 codes [2F, H] (scales [2F]); g as in h3_ffn_up. */
+H3_API h3_status h3_ffn_up_e4m3(const h3_dims* dims, h3_layout_t layout, int B,
+                                const void* h2_codes, const float* h2_scales, const void* w_codes,
+                                const float* w_scales, void* g, h3_stream_t stream);
+
 /* Workspace bytes of h3_block_forward_e4m3: h3_workspace_size plus the codes
  * [B*S, H] and scales [B*S] of the activation rows. */
 H3_API size_t h3_workspace_size_e4m3(const h3_dims* dims, int B, int S);

@@ -182,9 +182,17 @@ def split_w13(w13: np.ndarray, ffn: int) -> Tuple[np.ndarray, np.ndarray]:
 def qkv_project(h: np.ndarray, pos: np.ndarray, w_qkv: np.ndarray, q_norm: np.ndarray,
                 k_norm: np.ndarray, dims, emulate: bool = False,
                 need_q: bool = True) -> Tuple[Optional[np.ndarray], np.ndarray, np.ndarray]:
-    """h [n, H] -> q, k, v [n, NH, D] after QK-norm and RoPE (q, k only)."""
+    """h [n, H] -> q, k, v [n, NH, D] after QK-norm and RoPE (q, k only); w_qkv
+    as bf16 bits."""
+    return qkv_project_values(h, pos, bf16_to_f64(w_qkv), q_norm, k_norm, dims, emulate, need_q)
+
+
+def qkv_project_values(h: np.ndarray, pos: np.ndarray, w_qkv: np.ndarray, q_norm: np.ndarray,
+                       k_norm: np.ndarray, dims, emulate: bool = False,
+                       need_q: bool = True) -> Tuple[Optional[np.ndarray], np.ndarray, np.ndarray]:
+    """qkv_project with the weight [3 NH D, H] given as values."""
     NH, D = dims.heads, dims.head_dim
-    wq, wk, wv = split_qkv_weight(bf16_to_f64(w_qkv), NH, D)
+    wq, wk, wv = split_qkv_weight(np.asarray(w_qkv, F), NH, D)
     inv = rope_inv_freq(dims.rope_freq_dim, dims.rope_theta)
     qn, kn = bf16_to_f64(q_norm), bf16_to_f64(k_norm)
     n = h.shape[0]
@@ -235,8 +243,13 @@ def out_project_residual(x: np.ndarray, o: np.ndarray, gate: np.ndarray, w_o: np
 
 
 def ffn_gate(h2: np.ndarray, w13: np.ndarray, ffn: int, emulate: bool = False) -> np.ndarray:
-    """g = SiLU(h2 W1^T) * (h2 W3^T)."""
-    w1, w3 = split_w13(bf16_to_f64(w13), ffn)
+    """g = SiLU(h2 W1^T) * (h2 W3^T); w13 as bf16 bits."""
+    return ffn_gate_values(h2, bf16_to_f64(w13), ffn, emulate)
+
+
+def ffn_gate_values(h2: np.ndarray, w13: np.ndarray, ffn: int, emulate: bool = False) -> np.ndarray:
+    """ffn_gate with W1 || W3 [2F, H] given as values."""
+    w1, w3 = split_w13(np.asarray(w13, F), ffn)
     return _store(silu(h2 @ w1.T) * (h2 @ w3.T), emulate)
 
 
@@ -255,18 +268,28 @@ def _pre_attention(x, m, pos, w, dims, emulate, need_q=True):
     return qkv_project(h, pos, w.w_qkv, w.q_norm, w.k_norm, dims, emulate, need_q)
 
 
-def _post_attention(x, o, m, w, dims, emulate):
-    x1 = out_project_residual(x, o, m[:, 2], w.w_o, emulate)
+def _stream(a: np.ndarray, emulate: bool, stream_f32: bool) -> np.ndarray:
+    """Storage of the residual stream x1 / x2 under the emulation: bf16, or fp32
+    where the stream is held in fp32 (the stack's residual stream)."""
+    if emulate and stream_f32:
+        return np.asarray(a, np.float32).astype(F)
+    return _store(a, emulate)
+
+
+def _post_attention(x, o, m, w, dims, emulate, stream_f32=False):
+    x1 = _stream(out_project_residual(x, o, m[:, 2], w.w_o), emulate, stream_f32)
     h2 = _store(norm_modulate(x1, m[:, 3], m[:, 4], dims.norm_eps), emulate)
     g = ffn_gate(h2, w.w13, dims.ffn, emulate)
-    return ffn_down_residual(x1, g, m[:, 5], w.w2, emulate)
+    return _stream(ffn_down_residual(x1, g, m[:, 5], w.w2), emulate, stream_f32)
 
 
 def block_forward(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
-                  emulate: bool = False) -> np.ndarray:
+                  emulate: bool = False, stream_f32: bool = False) -> np.ndarray:
     """One block over the packed sequence. x [B, S, H] (values) -> [B, S, H] float64.
 
-    Padding rows (tag -1) are returned unchanged.
+    Padding rows (tag -1) are returned unchanged. ``emulate`` rounds to bf16 at
+    the device's storage points; with ``stream_f32`` the residual stream (x1 and
+    the output) is held in fp32 instead, as a stack of blocks holds it.
     """
     x = np.asarray(x, F)
     tags = np.asarray(layout.tags)
@@ -278,7 +301,7 @@ def block_forward(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
     for b in range(x.shape[0]):
         q, k, v = _pre_attention(x[b], m, layout.pos, w, dims, emulate)
         o = attention(q, pad, k, v, pad, emulate)
-        y = _post_attention(x[b], o, m, w, dims, emulate)
+        y = _post_attention(x[b], o, m, w, dims, emulate, stream_f32)
         out[b] = np.where(pad[:, None], x[b], y)
     return out
 
@@ -520,6 +543,19 @@ def quantize_rows_e4m3(a: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     return e4m3_round((a32 / s[:, None]).astype(np.float32)), s
 
 
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Values of e4m3 code bytes: bit 7 the sign, bits 6-3 the exponent field e
+    (bias 7), bits 2-0 the mantissa m; e = 0 gives 2^-6 m/8, otherwise
+    2^(e-7) (1 + m/8); e = 15 with m = 7 is NaN (no infinities)."""
+    c = np.asarray(codes, np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(F)
+    mag = np.where(e == 0, 2.0 ** -6 * m / 8.0, 2.0 ** (e.astype(F) - 7.0) * (1.0 + m / 8.0))
+    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
 def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return np.asarray(codes, F) * np.asarray(scales, F)[:, None]
 
@@ -549,24 +585,15 @@ def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
     pad = tags < 0
     m = row_modulation(tags, layout.t_idx, w.ada_table, tmod)
     out = np.empty_like(x)
-    NH, D = dims.heads, dims.head_dim
-    inv = rope_inv_freq(dims.rope_freq_dim, dims.rope_theta)
     for b in range(x.shape[0]):
         h = norm_modulate(x[b], m[:, 0], m[:, 1], dims.norm_eps)
         hq = dequantize_rows(*quantize_rows_e4m3(h))
-        wqs, wks, wvs = split_qkv_weight(wq.w_qkv, NH, D)
-        n = h.shape[0]
-        q = _store(rope_apply(rms_norm((hq @ wqs.T).reshape(n, NH, D), bf16_to_f64(w.q_norm),
-                                       dims.qk_norm_eps), layout.pos, inv), emulate)
-        k = _store(rope_apply(rms_norm((hq @ wks.T).reshape(n, NH, D), bf16_to_f64(w.k_norm),
-                                       dims.qk_norm_eps), layout.pos, inv), emulate)
-        v = _store((hq @ wvs.T).reshape(n, NH, D), emulate)
+        q, k, v = qkv_project_values(hq, layout.pos, wq.w_qkv, w.q_norm, w.k_norm, dims, emulate)
         o = attention(q, pad, k, v, pad, emulate)
         x1 = out_project_residual(x[b], o, m[:, 2], w.w_o, emulate)
         h2 = norm_modulate(x1, m[:, 3], m[:, 4], dims.norm_eps)
         h2q = dequantize_rows(*quantize_rows_e4m3(h2))
-        w1, w3 = split_w13(wq.w13, dims.ffn)
-        g = _store(silu(h2q @ w1.T) * (h2q @ w3.T), emulate)
+        g = ffn_gate_values(h2q, wq.w13, dims.ffn, emulate)
         y = ffn_down_residual(x1, g, m[:, 5], w.w2, emulate)
         out[b] = np.where(pad[:, None], x[b], y)
     return out

@@ -14,6 +14,12 @@ query rows (each row's softmax runs over that row's scores), so the pieces,
 put back in place, give the same result.
 ``tests/test_golden_stack_script.py`` checks that on small cases.
 
+With ``--emulate`` it writes tests/golden/stack_config5_golden_bf16.npz: the
+same stack with the oracle's bf16 storage emulation at the block's operand
+storage points (h, q, k, v, P, o, h2, g) and the residual stream in fp32, as the
+stack holds it on the device: the result of an exactly rounded bf16 stack, which
+separates the rounding every bf16 implementation carries from the device's own.
+
 The stored file holds the sampled row indices, the rows' bf16 input and
 float64 output (stored as float32), and a SHA-256 digest over every input the
 stack reads (layout, timesteps, activations, the prologue weights and all 50
@@ -39,6 +45,7 @@ from workloads import FULL_DIMS, activations, block_weights, config_layout, prol
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 OUT = os.path.join(HERE, "stack_config5_golden.npz")
+OUT_BF16 = os.path.join(HERE, "stack_config5_golden_bf16.npz")
 N_BLOCKS = 50
 
 
@@ -128,8 +135,11 @@ def main() -> None:
     ap.add_argument("--workers", type=int, default=len(os.sched_getaffinity(0)),
                     help="attention pieces run at once")
     ap.add_argument("--blocks", type=int, default=N_BLOCKS)
-    ap.add_argument("--out", default=OUT)
+    ap.add_argument("--out", default=None)
+    ap.add_argument("--emulate", action="store_true",
+                    help="bf16 at the device's operand storage points, fp32 residual stream")
     args = ap.parse_args()
+    out = args.out or (OUT_BF16 if args.emulate else OUT)
 
     dims = FULL_DIMS
     L = config_layout(5)
@@ -149,12 +159,12 @@ def main() -> None:
     for i in range(args.blocks):
         w = block_weights(dims, 5, i)
         dig.add_block(w)
-        y = O.block_forward(y, w, L, tmod, dims)
+        y = O.block_forward(y, w, L, tmod, dims, emulate=args.emulate, stream_f32=args.emulate)
         print(f"block {i + 1}/{args.blocks}: {time.time() - t0:.0f} s", flush=True)
-    np.savez(args.out, rows=rows, x_in_bits=xb[0, rows], x_out=y[0, rows].astype(np.float32),
+    np.savez(out, rows=rows, x_in_bits=xb[0, rows], x_out=y[0, rows].astype(np.float32),
              n_blocks=np.int64(args.blocks), input_sha256=np.array(dig.hexdigest()),
              seconds=np.float64(time.time() - t0), cores=np.int64(len(os.sched_getaffinity(0))))
-    print("wrote", args.out, "digest", dig.hexdigest())
+    print("wrote", out, "digest", dig.hexdigest())
 
 
 if __name__ == "__main__":

@@ -1037,6 +1037,22 @@ def test_e4m3_rounding_matches_torch_and_the_format():
                                   [1.0, 1.25, 16.0, 20.0])
 
 
+def test_e4m3_decode_matches_torch_on_every_byte():
+    """All 256 code bytes against torch's float8_e4m3fn reinterpretation; every
+    finite code's value lies on the e4m3 grid (e4m3_round keeps it); the NaN
+    codes are 0x7F and 0xFF only; the largest finite value is 448."""
+    b = np.arange(256, dtype=np.uint8)
+    got = O.e4m3_decode(b)
+    ref = torch.from_numpy(b).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[fin], ref[fin])
+    assert set(np.nonzero(np.isnan(got))[0]) == {0x7F, 0xFF}
+    np.testing.assert_array_equal(O.e4m3_round(got[fin]), got[fin])
+    assert np.nanmax(got) == 448.0 and O.e4m3_decode(np.array([1]))[0] == 2.0 ** -9
+    assert np.signbit(O.e4m3_decode(np.array([0x80]))[0])
+
+
 def test_row_quantization_round_trip():
     g = np.random.default_rng(9)
     a = (g.standard_normal((7, 300)) * np.array([1e-3, 1, 30, 0, 5, 1e4, 2])[:, None])

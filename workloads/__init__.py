@@ -31,4 +31,6 @@ from .h3_workloads import (  # noqa: F401
     DenoiserWeights,
     denoiser_weights,
     denoiser_inputs,
+    random_code_bytes,
+    random_scales,
 )

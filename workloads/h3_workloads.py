@@ -201,6 +201,21 @@ def uniform_f32(shape: Tuple[int, ...], seed: Sequence[int]) -> np.ndarray:
     return g.random(shape, dtype=np.float32)
 
 
+def random_code_bytes(shape: Tuple[int, ...], seed: Sequence[int]) -> np.ndarray:
+    """Uniform random bytes, excluding 0x7F and 0xFF (the two NaN codes of the
+    8-bit e4m3 format): operands for the 8-bit GEMM steps."""
+    g = np.random.default_rng(list(seed))
+    b = g.integers(0, 254, size=shape, dtype=np.int64)  # 254 values, then skip 0x7F
+    b = np.where(b >= 0x7F, b + 1, b)
+    return b.astype(np.uint8)
+
+
+def random_scales(n: int, seed: Sequence[int], lo: float = -12.0, hi: float = -6.0) -> np.ndarray:
+    """n positive float32 scales 2^u, u uniform in [lo, hi)."""
+    g = np.random.default_rng(list(seed))
+    return np.exp2(g.uniform(lo, hi, size=n)).astype(np.float32)
+
+
 # --------------------------------------------------------------------------
 # Packed layouts
 # --------------------------------------------------------------------------
