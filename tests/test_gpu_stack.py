@@ -22,6 +22,8 @@ pytestmark = pytest.mark.gpu
 
 GOLDEN5 = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
                        "stack_config5_golden.npz")
+GOLDEN5_BF16 = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                            "stack_config5_golden_bf16.npz")
 
 
 def gpu_stack(dl, dws, tmod, x, B):
@@ -135,32 +137,56 @@ def config5():
                 tmod=gpu_tmod(dims, L.timestep, pw), digest=dig.hexdigest())
 
 
+def _golden(path, config5):
+    g = np.load(path)
+    assert str(g["input_sha256"]) == config5["digest"], "inputs differ from the golden's"
+    assert int(g["n_blocks"]) == 50
+    np.testing.assert_array_equal(g["x_in_bits"], config5["xb"][0, g["rows"]])
+    return g
+
+
+def _stack_rows(config5, rows):
+    x = dev_bf16(config5["xb"])
+    gpu_stack(config5["dl"], config5["dws"], config5["tmod"], x, 1)
+    return host_f64(x[0, torch.from_numpy(rows).cuda()])
+
+
 def test_stack_config5_50_blocks_against_float64_golden(config5):
     """The full-width 50-block stack over the 16384-row padded layout against
     the float64 oracle's 50-block forward, stored at sampled rows by
     tests/golden/make_stack_config5_golden.py (rows next to every padding run,
-    in the mixed tiles, at tile edges, and random rows of each modality):
-    x_out and the stack's update x_out - x_in within rel-L2 1e-2 and max-abs
-    5e-2, padding rows bit-identical."""
-    g = np.load(GOLDEN5)
-    assert str(g["input_sha256"]) == config5["digest"], "inputs differ from the golden's"
-    assert int(g["n_blocks"]) == 50
+    in the mixed tiles, at tile edges, and random rows of each modality).
+
+    Against the float64 golden: x_out and the stack's update x_out - x_in within
+    rel-L2 1e-2; padding rows bit-identical. Against the oracle's bf16-storage
+    golden of the same stack (bf16 at every operand the device stores in bf16,
+    the residual stream in fp32, as on the device): rel-L2 1e-2 and max-abs 5e-2
+    beyond the output's own bf16 rounding. The largest difference from the
+    float64 golden is held to 5e-2 plus the distance between the two goldens:
+    after 50 blocks the residual stream reaches |x| ~ 20, where the bf16 operand
+    roundings that any bf16 stack performs move the output by more than 5e-2."""
+    g = _golden(GOLDEN5, config5)
     L, xb = config5["L"], config5["xb"]
     rows = g["rows"]
-    np.testing.assert_array_equal(g["x_in_bits"], xb[0, rows])
-    x = dev_bf16(xb)
-    gpu_stack(config5["dl"], config5["dws"], config5["tmod"], x, 1)
-    got = host_f64(x[0, torch.from_numpy(rows).cuda()])
+    got = _stack_rows(config5, rows)
     ref = g["x_out"].astype(np.float64)
     x0 = O.bf16_to_f64(xb[0, rows])
     pad = (L.tags < 0)[rows]
     assert pad.sum() >= 7 and (~pad).sum() >= 50
-    assert_close(got, ref, what="cfg5 50-block x_out")
+    assert_close(got, ref, what="cfg5 50-block x_out", mabs=np.inf)
     assert_close(got[~pad] - x0[~pad], ref[~pad] - x0[~pad], what="cfg5 50-block update",
                  mabs=np.inf)
     np.testing.assert_array_equal(got[pad], x0[pad])
     # the stack moved the valid rows far beyond bf16 resolution
     assert np.linalg.norm(ref[~pad] - x0[~pad]) > 0.5 * np.linalg.norm(x0[~pad])
+    gb = _golden(GOLDEN5_BF16, config5)
+    np.testing.assert_array_equal(gb["rows"], rows)
+    ref16 = gb["x_out"].astype(np.float64)
+    assert_close(got, ref16, what="cfg5 50-block x_out vs bf16-storage golden",
+                 storage_rounding=True)
+    spread = float(np.max(np.abs(ref16 - ref)))
+    d = float(np.max(np.abs(got - ref)))
+    assert d <= 5e-2 + spread, f"max-abs {d:.3e} vs float64 golden > 5e-2 + {spread:.3e}"
 
 
 def test_stack_config5_50_blocks_properties(config5):
