@@ -122,9 +122,7 @@ h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutVie
   e.L = L;
   e.B = B;
   e.NH = d.heads;
-  e.q = ws.q;
-  e.k = ws.k;
-  e.v = ws.v;
+  e.heads = plain_head_map(ws.q, ws.k, ws.v, d.heads, L.S);
   e.q_norm = w.q_norm;
   e.k_norm = w.k_norm;
   e.qk_eps = d.qk_norm_eps;
@@ -415,9 +413,7 @@ h3_status h3_qkv_rope(const h3_dims* dims, h3_layout_t L, int B, const void* h, 
   e.L = L->view();
   e.B = B;
   e.NH = dims->heads;
-  e.q = q;
-  e.k = k;
-  e.v = v;
+  e.heads = plain_head_map(q, k, v, dims->heads, L->S);
   e.q_norm = q_norm;
   e.k_norm = k_norm;
   e.qk_eps = dims->qk_norm_eps;
@@ -789,6 +785,87 @@ h3_status h3_stack_forward_reduced(const h3_dims* dims, const h3_block_weights* 
 
 }  // extern "C"
 
+// ---- sequence-parallel block: exchanges fused into the producing kernels ----
+
+namespace {
+
+h3_status check_peers(const h3_dims* dims, const h3_ulysses_peers* p, int S_full) {
+  if (!p) return H3_ERR_ARG;
+  const int P = p->n_ranks;
+  if (P < 1 || P > H3_MAX_RANKS || H3_MAX_RANKS > kMaxDst || p->rank < 0 || p->rank >= P)
+    return H3_ERR_ARG;
+  if (dims->heads % P != 0 || S_full % P != 0) return H3_ERR_SHAPE;
+  return H3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+h3_status h3_qkv_rope_to_heads(const h3_dims* dims, h3_layout_t chunk, const void* h,
+                               const void* w_qkv, const void* q_norm, const void* k_norm,
+                               const h3_ulysses_peers* peers, h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!chunk || !h || !w_qkv || !q_norm || !k_norm || !peers) return H3_ERR_ARG;
+  H3_TRY(check_batch(chunk, 1));
+  const int P = peers->n_ranks;
+  if (P < 1 || P > H3_MAX_RANKS) return H3_ERR_ARG;
+  const long long S_full = (long long)chunk->S * P;
+  if (S_full > kMaxRows) return H3_ERR_SHAPE;
+  H3_TRY(check_peers(dims, peers, (int)S_full));
+  if (!aligned16(h) || !aligned16(w_qkv) || !aligned16(q_norm) || !aligned16(k_norm))
+    return H3_ERR_ALIGN;
+  for (int j = 0; j < P; ++j) {
+    if (!peers->q[j] || !peers->k[j] || !peers->v[j]) return H3_ERR_ARG;
+    if (!aligned16(peers->q[j]) || !aligned16(peers->k[j]) || !aligned16(peers->v[j]))
+      return H3_ERR_ALIGN;
+  }
+  GemmEpiArgs e;
+  e.L = chunk->view();
+  e.B = 1;
+  e.NH = dims->heads;
+  for (int j = 0; j < P; ++j) {
+    e.heads.q[j] = peers->q[j];
+    e.heads.k[j] = peers->k[j];
+    e.heads.v[j] = peers->v[j];
+  }
+  e.heads.heads_per_dst = dims->heads / P;
+  e.heads.dst_rows = (int)S_full;
+  e.heads.row_offset = peers->rank * chunk->S;
+  e.q_norm = q_norm;
+  e.k_norm = k_norm;
+  e.qk_eps = dims->qk_norm_eps;
+  H3_CUDA(launch_gemm(EPI_QKV, chunk->S, 3 * dims->heads * dims->head_dim, dims->hidden, h, w_qkv,
+                      e, as_stream(stream)));
+  return H3_OK;
+}
+
+h3_status h3_attention_to_rows(const h3_dims* dims, h3_layout_t full, const void* q,
+                               const void* k, const void* v, const h3_ulysses_peers* peers,
+                               h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!full || !q || !k || !v || !peers) return H3_ERR_ARG;
+  H3_TRY(check_batch(full, 1));
+  H3_TRY(check_peers(dims, peers, full->S));
+  const int P = peers->n_ranks;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return H3_ERR_ALIGN;
+  for (int j = 0; j < P; ++j) {
+    if (!peers->o[j]) return H3_ERR_ARG;
+    if (!aligned16(peers->o[j])) return H3_ERR_ALIGN;
+  }
+  const int NHl = dims->heads / P;
+  RowMap m;
+  for (int j = 0; j < P; ++j) m.o[j] = peers->o[j];
+  m.rows_per_dst = full->S / P;
+  m.row_heads = dims->heads;
+  m.head_offset = peers->rank * NHl;
+  if (full->S == 0) return H3_OK;
+  H3_CUDA(launch_attention(full->view(), 1, NHl, q, k, v, m, as_stream(stream)));
+  return H3_OK;
+}
+
+}  // extern "C"
+
 // ---- 8-bit QKV and W1 || W3 GEMM inputs ----
 
 extern "C" {
@@ -837,9 +914,7 @@ h3_status h3_qkv_rope_e4m3(const h3_dims* dims, h3_layout_t L, int B, const void
   e.L = L->view();
   e.B = B;
   e.NH = dims->heads;
-  e.q = q;
-  e.k = k;
-  e.v = v;
+  e.heads = plain_head_map(q, k, v, dims->heads, L->S);
   e.q_norm = q_norm;
   e.k_norm = k_norm;
   e.qk_eps = dims->qk_norm_eps;

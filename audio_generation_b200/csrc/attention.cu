@@ -135,10 +135,17 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
+// Start of the 128 output values of row s, head h of batch element b.
+__device__ __forceinline__ __nv_bfloat16* out_row(const RowMap& m, int b, int s, int h) {
+  const int g = s / m.rows_per_dst, sl = s - g * m.rows_per_dst;
+  return reinterpret_cast<__nv_bfloat16*>(m.o[g]) +
+         (((size_t)b * m.rows_per_dst + sl) * m.row_heads + m.head_offset + h) * D;
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_attention(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const LayoutView L, int NH,
-                __nv_bfloat16* __restrict__ o, float scale_log2) {
+                const __grid_constant__ RowMap om, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -159,7 +166,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (threadIdx.x < 256) {
       const int s = q0 + threadIdx.x;
       if (s < S) {
-        uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * S + s) * NH + head) * D);
+        uint4* dst = reinterpret_cast<uint4*>(out_row(om, b, s, head));
 #pragma unroll
         for (int i = 0; i < 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
       }
@@ -438,7 +445,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool tile_pad = i == 0 ? pad0 : pad1;
     const bool row_ok = ok && s < S;
     const float inv_l = (l_run > 0.f && !tile_pad) ? 1.f / l_run : 0.f;
-    __nv_bfloat16* dst = o + (((size_t)b * S + (row_ok ? s : 0)) * NH + head) * D;
+    __nv_bfloat16* dst = out_row(om, b, row_ok ? s : 0, head);
     uint32_t rr[32];
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
@@ -470,7 +477,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }  // namespace
 
 cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, const void* k,
-                             const void* v, void* o, cudaStream_t st) {
+                             const void* v, const RowMap& out, cudaStream_t st) {
   if (L.S == 0 || B == 0) return cudaSuccess;
   if (L.n_tiles > kMaxKeyTiles || B > kMaxBatch) return cudaErrorInvalidValue;
   cudaError_t err =
@@ -486,9 +493,9 @@ cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, 
     return cudaErrorInvalidValue;
   const float scale_log2 = 1.4426950408889634f / 11.313708498984761f;  // log2(e) / sqrt(128)
   dim3 grid((L.n_tiles + 1) / 2, NH, B);
-  k_attention<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tq, tk, tv, L, NH,
-                                                     reinterpret_cast<__nv_bfloat16*>(o),
-                                                     scale_log2);
+  if (out.rows_per_dst <= 0 || (L.S + out.rows_per_dst - 1) / out.rows_per_dst > kMaxDst)
+    return cudaErrorInvalidValue;
+  k_attention<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tq, tk, tv, L, NH, out, scale_log2);
   return cudaGetLastError();
 }
 

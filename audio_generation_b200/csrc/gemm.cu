@@ -208,9 +208,11 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
       const int u = n0 / 128 + su;
       const int head = u / 3, kind = u % 3;
       const uint32_t tbase = taddr + 128 * su;
+      const HeadMap& hm = e.heads;
+      const int g = head / hm.heads_per_dst, lh = head - g * hm.heads_per_dst;
       __nv_bfloat16* dst =
-          reinterpret_cast<__nv_bfloat16*>(kind == 0 ? e.q : (kind == 1 ? e.k : e.v)) +
-          (((size_t)b * e.NH + head) * S + s) * 128;
+          reinterpret_cast<__nv_bfloat16*>(kind == 0 ? hm.q[g] : (kind == 1 ? hm.k[g] : hm.v[g])) +
+          (((size_t)b * hm.heads_per_dst + lh) * hm.dst_rows + hm.row_offset + s) * 128;
       const float* sw = e.b_scale + n0 + 128 * su;
       if (kind == 2) {
 #pragma unroll 1
@@ -277,7 +279,7 @@ constexpr int p_smem_bytes() { return PNST * p_stage<BN>() + 1024 + 256; }
 template <int EPI, int BN, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                int M, int N, int K, int group_n, const GemmEpiArgs e) {
+                int M, int N, int K, int group_n, const __grid_constant__ GemmEpiArgs e) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

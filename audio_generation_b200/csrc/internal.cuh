@@ -138,13 +138,55 @@ enum GemmEpilogue {
   EPI_F32 = 5
 };
 
+// Up to this many destination buffers for the outputs of one launch (the ranks
+// of the sequence-parallel block; one for the plain block).
+constexpr int kMaxDst = 8;
+
+// Where EPI_QKV puts q / k / v of head h, row s of batch element b:
+// q[h / heads_per_dst] + ((b * heads_per_dst + h % heads_per_dst) * dst_rows
+// + row_offset + s) * 128 (likewise k, v). The plain block: one destination
+// with all NH heads, dst_rows = S, row_offset = 0.
+struct HeadMap {
+  void* q[kMaxDst] = {};
+  void* k[kMaxDst] = {};
+  void* v[kMaxDst] = {};
+  int heads_per_dst = 0, dst_rows = 0, row_offset = 0;
+};
+
+// Where attention puts the output of row s, head h (of this launch's NH heads)
+// of batch element b: o[s / rows_per_dst] + ((b * rows_per_dst + s %
+// rows_per_dst) * row_heads + head_offset + h) * 128. The plain block: one
+// destination, rows_per_dst = S, row_heads = NH, head_offset = 0.
+struct RowMap {
+  void* o[kMaxDst] = {};
+  int rows_per_dst = 0, row_heads = 0, head_offset = 0;
+};
+
+inline HeadMap plain_head_map(void* q, void* k, void* v, int NH, int S) {
+  HeadMap m;
+  m.q[0] = q;
+  m.k[0] = k;
+  m.v[0] = v;
+  m.heads_per_dst = NH;
+  m.dst_rows = S;
+  return m;
+}
+
+inline RowMap plain_row_map(void* o, int NH, int S) {
+  RowMap m;
+  m.o[0] = o;
+  m.rows_per_dst = S;
+  m.row_heads = NH;
+  return m;
+}
+
 struct GemmEpiArgs {
   LayoutView L;
   int B = 1, NH = 0;
   // EPI_STORE: out [M, N] bf16; EPI_F32: out [M, N] fp32; EPI_SWIGLU: out [M, N/2]
   void* out = nullptr;
   // EPI_QKV
-  void *q = nullptr, *k = nullptr, *v = nullptr;
+  HeadMap heads;
   const void *q_norm = nullptr, *k_norm = nullptr;
   float qk_eps = 0.f;
   // EPI_RESID: x [M, N] in/out, gate = table[tag][gate_chunk] + tmod[t_idx][gate_chunk]
@@ -167,7 +209,11 @@ cudaError_t launch_gemm_e4m3(int epi, int M, int N, int K, const void* A, const 
                              const GemmEpiArgs& e, cudaStream_t st);
 
 cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q, const void* k,
-                             const void* v, void* o, cudaStream_t st);
+                             const void* v, const RowMap& out, cudaStream_t st);
+inline cudaError_t launch_attention(const LayoutView& L, int B, int NH, const void* q,
+                                    const void* k, const void* v, void* o, cudaStream_t st) {
+  return launch_attention(L, B, NH, q, k, v, plain_row_map(o, NH, L.S), st);
+}
 
 int num_sms();
 

@@ -71,6 +71,15 @@ class h3_block_weights_e4m3(ctypes.Structure):
         "w_qkv_codes", "w_qkv_scales", "w13_codes", "w13_scales")]
 
 
+H3_MAX_RANKS = 8
+
+
+class h3_ulysses_peers(ctypes.Structure):
+    _fields_ = [("n_ranks", ctypes.c_int), ("rank", ctypes.c_int),
+                ("q", ctypes.c_void_p * H3_MAX_RANKS), ("k", ctypes.c_void_p * H3_MAX_RANKS),
+                ("v", ctypes.c_void_p * H3_MAX_RANKS), ("o", ctypes.c_void_p * H3_MAX_RANKS)]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -102,6 +111,10 @@ _SIGNATURES = {
     "h3_block_forward": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights), _vp,
                               _vp, _vp, _i, _vp, _sz, _vp]),
     "h3_quantize_e4m3_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "h3_qkv_rope_to_heads": (_i, [ctypes.POINTER(h3_dims), _vp, _vp, _vp, _vp, _vp,
+                                  ctypes.POINTER(h3_ulysses_peers), _vp]),
+    "h3_attention_to_rows": (_i, [ctypes.POINTER(h3_dims), _vp, _vp, _vp, _vp,
+                                  ctypes.POINTER(h3_ulysses_peers), _vp]),
     "h3_norm_modulate_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _i, _vp, _vp, _vp, _vp,
                                    _vp, _vp]),
     "h3_qkv_rope_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -399,6 +412,34 @@ def h3_stack_forward_reduced(dims: h3_dims, weights: Sequence[h3_block_weights],
 def h3_quantize_e4m3_rows(w, rows: int, K: int, codes, scales, stream=None) -> None:
     _check(lib().h3_quantize_e4m3_rows(_ptr(w), rows, K, _ptr(codes), _ptr(scales),
                                        _stream(stream)), "h3_quantize_e4m3_rows")
+
+
+def make_peers(rank: int, q, k, v, o) -> h3_ulysses_peers:
+    """The exchange destinations of one rank: q, k, v, o are per-rank lists of
+    tensors or raw device addresses (ints), one entry per rank."""
+    P = len(q)
+    if not (len(k) == len(v) == len(o) == P) or not 1 <= P <= H3_MAX_RANKS:
+        raise ValueError("one q, k, v and o destination per rank, at most %d ranks" % H3_MAX_RANKS)
+    addr = lambda t: t if isinstance(t, int) else _ptr(t)
+    p = h3_ulysses_peers()
+    p.n_ranks, p.rank = P, rank
+    for j in range(P):
+        p.q[j], p.k[j], p.v[j], p.o[j] = addr(q[j]), addr(k[j]), addr(v[j]), addr(o[j])
+    return p
+
+
+def h3_qkv_rope_to_heads(dims: h3_dims, chunk: Layout, h, w_qkv, q_norm, k_norm,
+                         peers: h3_ulysses_peers, stream=None) -> None:
+    _check(lib().h3_qkv_rope_to_heads(ctypes.byref(dims), chunk.handle, _ptr(h), _ptr(w_qkv),
+                                      _ptr(q_norm), _ptr(k_norm), ctypes.byref(peers),
+                                      _stream(stream)), "h3_qkv_rope_to_heads")
+
+
+def h3_attention_to_rows(dims: h3_dims, full: Layout, q, k, v, peers: h3_ulysses_peers,
+                         stream=None) -> None:
+    _check(lib().h3_attention_to_rows(ctypes.byref(dims), full.handle, _ptr(q), _ptr(k), _ptr(v),
+                                      ctypes.byref(peers), _stream(stream)),
+           "h3_attention_to_rows")
 
 
 def h3_norm_modulate_e4m3(dims: h3_dims, layout: Layout, B: int, which: int, x, ada_table, tmod,

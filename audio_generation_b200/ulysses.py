@@ -14,13 +14,24 @@ document is the same), and a second all-to-all turns the output back into "my
 rows, all heads".
 
 Every step runs in this library's kernels through the C ABI; this module only
-allocates, reshapes and exchanges buffers. The exchange is a callable
-``all_to_all(out, inp)`` that splits dim 0 of ``inp`` evenly across ranks, as
-``torch.distributed.all_to_all_single`` does (NCCL over NVLink between GPUs).
-The three stages of :class:`UlyssesBlock` are public so that the exchange can
-also be carried out by a caller that holds every rank's buffers.
+allocates, reshapes and exchanges buffers. Two forms of the exchange:
 
-Requirements: S % P == 0 and heads % P == 0.
+* fused (``forward_fused``): the QKV kernel's epilogue stores each head's rows
+  straight into the receive buffer of the rank that owns the head
+  (h3_qkv_rope_to_heads), and the attention kernel stores each row's output
+  straight into the receive buffer of the rank that owns the row
+  (h3_attention_to_rows). The receive buffers are this GPU's or peers' memory
+  (``symmetric_receive_buffers`` maps them through torch's symmetric memory);
+  the ranks only synchronise between the phases (``barrier``). No copy or
+  collective runs on the data path.
+* through a callable ``all_to_all(out, inp)`` that splits dim 0 of ``inp``
+  evenly across ranks, as ``torch.distributed.all_to_all_single`` (NCCL) does
+  (``forward``).
+
+The stages of :class:`UlyssesBlock` are public so that a caller that holds every
+rank's buffers (one process, one GPU) can run the ranks in turn.
+
+Requirements: S % P == 0, heads % P == 0 and P <= 8 for the fused form.
 """
 
 from __future__ import annotations
@@ -72,7 +83,7 @@ class UlyssesBlock:
     """
 
     def __init__(self, dims, layout, rank: int, world: int, device,
-                 all_to_all: Optional[Callable] = None):
+                 all_to_all: Optional[Callable] = None, receive=None):
         S, NH = layout.S, dims.heads
         if S % world or NH % world:
             raise ValueError("the sequence length and the head count must divide by the ranks")
@@ -95,6 +106,12 @@ class UlyssesBlock:
         self.q, self.k, self.v = bf(1, NH, self.Sr, D), bf(1, NH, self.Sr, D), bf(1, NH, self.Sr, D)
         self.ol = bf(1, S, self.NHl * D)
         self.g = bf(1, self.Sr, F)
+        # receive buffers of the fused exchange: q, k, v [NH / P, S, D] (every
+        # row of this rank's heads) and o [S / P, NH D] (this rank's rows)
+        if receive is None:
+            receive = (bf(self.NHl, S, D), bf(self.NHl, S, D), bf(self.NHl, S, D),
+                       bf(self.Sr, NH * D))
+        self.recv = receive
 
     def pre_attention(self, w, tmod, x):
         """norm1 + modulate and QKV + QK-norm + RoPE on this rank's rows: x [1, Sr, H]."""
@@ -116,6 +133,28 @@ class UlyssesBlock:
         h3.h3_ffn_up(self.d, self.chunk, 1, self.h, w.w13, self.g)
         h3.h3_ffn_down_residual(self.d, self.chunk, 1, self.g, w.w2, w.ada_table, tmod, x)
 
+    def pre_attention_to_heads(self, w, tmod, x, peers):
+        """norm1 + modulate on this rank's rows, then QKV + QK-norm + RoPE with
+        every head's rows stored into its owner's receive buffer."""
+        h3.h3_norm_modulate(self.d, self.chunk, 1, 0, x, w.ada_table, tmod, self.h)
+        h3.h3_qkv_rope_to_heads(self.d, self.chunk, self.h, w.w_qkv, w.q_norm, w.k_norm, peers)
+
+    def attention_to_rows(self, peers):
+        """Attention of this rank's heads over every row (its receive buffers),
+        every row's output stored into its owner's receive buffer."""
+        q, k, v, _ = self.recv
+        h3.h3_attention_to_rows(self.d, self.full, q, k, v, peers)
+
+    def forward_fused(self, w, tmod, x, peers, barrier: Callable):
+        """The whole block with the fused exchange; ``barrier()`` orders the
+        phases across ranks (every rank's stores complete before any rank reads
+        them)."""
+        self.pre_attention_to_heads(w, tmod, x, peers)
+        barrier()
+        self.attention_to_rows(peers)
+        barrier()
+        self.post_attention(w, tmod, self.recv[3][None], x)
+
     def forward(self, w, tmod, x):
         """The whole block on this rank's rows, exchanging with the other ranks."""
         if self.all_to_all is None:
@@ -128,6 +167,58 @@ class UlyssesBlock:
     def close(self):
         self.full.close()
         self.chunk.close()
+
+
+def receive_shapes(dims, S: int, world: int):
+    """Shapes of one rank's q, k, v and o receive buffers (bf16)."""
+    NHl, D = dims.heads // world, dims.head_dim
+    return [(NHl, S, D)] * 3 + [(S // world, dims.heads * D)]
+
+
+def receive_offsets(dims, S: int, world: int):
+    """Byte offsets of q, k, v and o inside one rank's receive area, each
+    256-byte aligned, and the area's size."""
+    offs, at = [], 0
+    for shp in receive_shapes(dims, S, world):
+        offs.append(at)
+        n = 2
+        for d in shp:
+            n *= d
+        at += (n + 255) // 256 * 256
+    return offs, at
+
+
+def symmetric_receive_buffers(dims, S: int, group=None):
+    """Receive buffers in torch's symmetric memory, one area per rank at the
+    same offsets: returns (this rank's q, k, v, o views, the peers of every
+    rank's areas as lists of addresses (q, k, v, o), the handle)."""
+    import torch.distributed as dist
+    import torch.distributed._symmetric_memory as symm_mem
+
+    world = dist.get_world_size(group)
+    offs, size = receive_offsets(dims, S, world)
+    area = symm_mem.empty(size, dtype=torch.uint8, device=torch.device("cuda",
+                                                                       torch.cuda.current_device()))
+    hdl = symm_mem.rendezvous(area, group if group is not None else dist.group.WORLD)
+    views = []
+    for off, shp in zip(offs, receive_shapes(dims, S, world)):
+        n = 1
+        for d in shp:
+            n *= d
+        views.append(area[off:off + 2 * n].view(torch.bfloat16).view(*shp))
+    ptrs = [int(p) for p in hdl.buffer_ptrs]
+    lists = [[p + off for p in ptrs] for off in offs]
+    return tuple(views), lists, hdl
+
+
+def host_barrier(group=None) -> Callable:
+    """Phase barrier between ranks: this GPU's work done, then the ranks meet."""
+    import torch.distributed as dist
+
+    def barrier():
+        torch.cuda.current_stream().synchronize()
+        dist.barrier(group=group)
+    return barrier
 
 
 def nccl_all_to_all(group=None) -> Callable:

@@ -282,6 +282,48 @@ H3_API h3_status h3_stack_forward(const h3_dims* dims, const h3_block_weights* w
                            h3_layout_t layout, const float* tmod, void* x, int B, void* ws,
                            size_t ws_bytes, h3_stream_t stream);
 
+/* ---- sequence-parallel block: the head <-> sequence exchange fused into the
+ * kernels that produce the exchanged tensors ---- */
+
+/* "MiniMaxH3Transformer3DModel" page, `forward`: each batch element is one
+ * attention document over one packed sequence, so one long sequence is split
+ * across P ranks by rows. Every step but attention is row-local; attention is
+ * independent per head. Rank r holds rows [r S/P, (r + 1) S/P) (its chunk) and,
+ * for attention, heads [r NH/P, (r + 1) NH/P) of every row.
+ *
+ * The two exchanges are stores from the producing kernels into the receiving
+ * rank's buffer: plain global stores, so a buffer may be another GPU's memory
+ * mapped into this process (peer access over NVLink) or, with every rank in one
+ * process, a buffer of this GPU. These calls only enqueue; the caller orders
+ * them across ranks (all ranks' h3_qkv_rope_to_heads complete before any
+ * rank's h3_attention_to_rows reads its q, k, v, and all ranks'
+ * h3_attention_to_rows complete before any rank reads its o). */
+#define H3_MAX_RANKS 8
+typedef struct {
+  int n_ranks; /* P, 1 .. H3_MAX_RANKS; S % P == 0 and heads % P == 0 */
+  int rank;    /* this rank, 0 .. P - 1 */
+  void* q[H3_MAX_RANKS]; /* rank j's q [heads / P, S, 128] bf16 (likewise k, v) */
+  void* k[H3_MAX_RANKS];
+  void* v[H3_MAX_RANKS];
+  void* o[H3_MAX_RANKS]; /* rank j's o [S / P, heads * 128] bf16 */
+} h3_ulysses_peers;
+
+/* h3_qkv_rope (B = 1) on this rank's chunk: `chunk` is the layout of its S / P
+ * rows (their positions drive RoPE), h [S/P, H]. Head n of chunk row s goes
+ * to rank n / (heads / P): q[..][n % (heads / P)][rank * S / P + s][:], and
+ * likewise k, v. */
+H3_API h3_status h3_qkv_rope_to_heads(const h3_dims* dims, h3_layout_t chunk, const void* h,
+                                      const void* w_qkv, const void* q_norm, const void* k_norm,
+                                      const h3_ulysses_peers* peers, h3_stream_t stream);
+
+/* h3_attention (B = 1) of this rank's heads / P heads over every row: `full` is
+ * the layout of all S rows, q, k, v [heads / P, S, 128] this rank's buffers
+ * (dims->heads is the total head count). The output of row s, local head n
+ * goes to rank s / (S / P): o[..][s % (S / P)][(rank * heads / P + n) * 128 ..]. */
+H3_API h3_status h3_attention_to_rows(const h3_dims* dims, h3_layout_t full, const void* q,
+                                      const void* k, const void* v,
+                                      const h3_ulysses_peers* peers, h3_stream_t stream);
+
 /* ---- 8-bit (e4m3) inputs for the QKV and W1 || W3 GEMMs ---- */
 
 /* "MiniMax H3 Inference Engine voor Mac computers", sections "Profiling en

@@ -58,3 +58,27 @@ def test_exchange_between_processes(world):
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(world))
     assert res == [(r, True, True) for r in range(world)]
+
+
+def test_fused_exchange_receive_areas_and_peer_table():
+    """Host side of the fused exchange: the receive areas hold q, k, v and o at
+    256-byte aligned offsets with the right sizes, and make_peers lays out one
+    destination per rank (raw addresses accepted) and rejects more than 8."""
+    from audio_generation_b200 import h3
+    from audio_generation_b200.ulysses import receive_offsets, receive_shapes
+    from workloads import FULL_DIMS
+
+    S, P = 16384, 8
+    shapes = receive_shapes(FULL_DIMS, S, P)
+    assert shapes == [(7, S, 128)] * 3 + [(S // 8, 7168)]
+    offs, size = receive_offsets(FULL_DIMS, S, P)
+    assert all(o % 256 == 0 for o in offs)
+    sizes = [2 * int(np.prod(s)) for s in shapes]
+    assert [b - a for a, b in zip(offs, offs[1:] + [size])] == sizes  # no gaps: all multiples of 256
+    base = [0x7f0000000000 + j * (1 << 32) for j in range(P)]
+    lists = [[b + o for b in base] for o in offs]
+    p = h3.make_peers(3, *lists)
+    assert p.n_ranks == 8 and p.rank == 3
+    assert [p.q[j] for j in range(P)] == lists[0] and [p.o[j] for j in range(P)] == lists[3]
+    with pytest.raises(ValueError):
+        h3.make_peers(0, *[[1] * 9] * 4)
