@@ -63,6 +63,15 @@ struct Workspace {
   void *q, *k, *v, *g;
 };
 
+// Bytes per row of the 8-bit activation codes: the widest GEMM input (h, o or g).
+size_t e4m3_row_bytes(const h3_dims& d) {
+  size_t m = (size_t)d.hidden;
+  const size_t A = (size_t)d.heads * d.head_dim;
+  if (A > m) m = A;
+  if ((size_t)d.ffn > m) m = d.ffn;
+  return m;
+}
+
 size_t ws_parts(const h3_dims& d, int B, int S, Workspace* w, void* base) {
   const size_t rows = (size_t)B * S;
   const size_t A = (size_t)d.heads * d.head_dim;
@@ -142,7 +151,15 @@ h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutVie
   r.tmod = tmod;
   r.gate_chunk = 2;
   const int resid = x_f32 ? EPI_RESID_F32 : EPI_RESID;
-  H3_CUDA(launch_gemm(resid, M, H, A, ws.o, w.w_o, r, st));
+  if (q8.w && q8.w->w_o_codes) {  // o as stored (bf16), quantized per row
+    H3_CUDA(launch_quantize_rows_e4m3(M, A, ws.o, q8.codes, q8.scales, st));
+    GemmEpiArgs r8 = r;
+    r8.a_scale = q8.scales;
+    r8.b_scale = q8.w->w_o_scales;
+    H3_CUDA(launch_gemm_e4m3(resid, M, H, A, q8.codes, q8.w->w_o_codes, r8, st));
+  } else {
+    H3_CUDA(launch_gemm(resid, M, H, A, ws.o, w.w_o, r, st));
+  }
   GemmEpiArgs sg;
   sg.L = L;
   sg.out = ws.g;
@@ -158,7 +175,15 @@ h3_status run_block(const h3_dims& d, const h3_block_weights& w, const LayoutVie
     H3_CUDA(launch_gemm(EPI_SWIGLU, M, 2 * Fd, H, ws.h, w.w13, sg, st));
   }
   r.gate_chunk = 5;
-  H3_CUDA(launch_gemm(resid, M, H, Fd, ws.g, w.w2, r, st));
+  if (q8.w && q8.w->w2_codes) {  // g as stored (bf16), quantized per row
+    H3_CUDA(launch_quantize_rows_e4m3(M, Fd, ws.g, q8.codes, q8.scales, st));
+    GemmEpiArgs r8 = r;
+    r8.a_scale = q8.scales;
+    r8.b_scale = q8.w->w2_scales;
+    H3_CUDA(launch_gemm_e4m3(resid, M, H, Fd, q8.codes, q8.w->w2_codes, r8, st));
+  } else {
+    H3_CUDA(launch_gemm(resid, M, H, Fd, ws.g, w.w2, r, st));
+  }
   return H3_OK;
 }
 
@@ -948,8 +973,61 @@ h3_status h3_ffn_up_e4m3(const h3_dims* dims, h3_layout_t L, int B, const void* 
 size_t h3_workspace_size_e4m3(const h3_dims* dims, int B, int S) {
   if (check_dims(dims) != H3_OK || B < 0 || S < 0) return 0;
   const size_t rows = (size_t)B * S;
-  return ws_parts(*dims, B, S, nullptr, nullptr) + align256(rows * dims->hidden) +
+  return ws_parts(*dims, B, S, nullptr, nullptr) + align256(rows * e4m3_row_bytes(*dims)) +
          align256(rows * 4);
+}
+
+}  // extern "C"
+
+namespace {
+
+h3_status resid_e4m3(const h3_dims* dims, h3_layout_t L, int B, int K, int gate_chunk,
+                     const void* a_codes, const float* a_scales, const void* w_codes,
+                     const float* w_scales, const float* ada_table, const float* tmod, void* x,
+                     h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || !a_codes || !a_scales || !w_codes || !w_scales || !ada_table || !tmod || !x)
+    return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(ada_table) || !aligned16(tmod) || !aligned16(x))
+    return H3_ERR_ALIGN;
+  if (dims->hidden % 256 != 0 || K % 128 != 0) return H3_ERR_SHAPE;
+  GemmEpiArgs r;
+  r.L = L->view();
+  r.B = B;
+  r.x = x;
+  r.table = ada_table;
+  r.tmod = tmod;
+  r.gate_chunk = gate_chunk;
+  r.a_scale = a_scales;
+  r.b_scale = w_scales;
+  H3_CUDA(launch_gemm_e4m3(EPI_RESID, B * L->S, dims->hidden, K, a_codes, w_codes, r,
+                           as_stream(stream)));
+  return H3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+h3_status h3_out_residual_e4m3(const h3_dims* dims, h3_layout_t L, int B, const void* o_codes,
+                               const float* o_scales, const void* w_codes, const float* w_scales,
+                               const float* ada_table, const float* tmod, void* x,
+                               h3_stream_t stream) {
+  if (!dims) return H3_ERR_ARG;
+  return resid_e4m3(dims, L, B, dims->heads * dims->head_dim, 2, o_codes, o_scales, w_codes,
+                    w_scales, ada_table, tmod, x, stream);
+}
+
+h3_status h3_ffn_down_residual_e4m3(const h3_dims* dims, h3_layout_t L, int B,
+                                    const void* g_codes, const float* g_scales,
+                                    const void* w_codes, const float* w_scales,
+                                    const float* ada_table, const float* tmod, void* x,
+                                    h3_stream_t stream) {
+  if (!dims) return H3_ERR_ARG;
+  return resid_e4m3(dims, L, B, dims->ffn, 5, g_codes, g_scales, w_codes, w_scales, ada_table,
+                    tmod, x, stream);
 }
 
 h3_status h3_block_forward_e4m3(const h3_dims* dims, const h3_block_weights* weights,
@@ -962,10 +1040,14 @@ h3_status h3_block_forward_e4m3(const h3_dims* dims, const h3_block_weights* wei
   H3_TRY(check_weights(weights));
   if (!w8->w_qkv_codes || !w8->w_qkv_scales || !w8->w13_codes || !w8->w13_scales)
     return H3_ERR_ARG;
+  if ((w8->w_o_codes && !w8->w_o_scales) || (w8->w2_codes && !w8->w2_scales)) return H3_ERR_ARG;
   if (!aligned16(w8->w_qkv_codes) || !aligned16(w8->w_qkv_scales) || !aligned16(w8->w13_codes) ||
-      !aligned16(w8->w13_scales) || !aligned16(tmod) || !aligned16(x) || !aligned16(ws))
+      !aligned16(w8->w13_scales) || !aligned16(w8->w_o_codes) || !aligned16(w8->w_o_scales) ||
+      !aligned16(w8->w2_codes) || !aligned16(w8->w2_scales) || !aligned16(tmod) ||
+      !aligned16(x) || !aligned16(ws))
     return H3_ERR_ALIGN;
   if (dims->hidden % 128 != 0) return H3_ERR_SHAPE;
+  if ((w8->w_o_codes || w8->w2_codes) && dims->hidden % 256 != 0) return H3_ERR_SHAPE;
   if (ws_bytes < h3_workspace_size_e4m3(dims, B, L->S)) return H3_ERR_WORKSPACE;
   Workspace w;
   const size_t base = ws_parts(*dims, B, L->S, &w, ws);
@@ -973,7 +1055,7 @@ h3_status h3_block_forward_e4m3(const h3_dims* dims, const h3_block_weights* wei
   q8.w = w8;
   q8.codes = static_cast<uint8_t*>(ws) + base;
   q8.scales = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + base +
-                                       align256((size_t)B * L->S * dims->hidden));
+                                       align256((size_t)B * L->S * e4m3_row_bytes(*dims)));
   return run_block(*dims, *weights, L->view(), tmod, x, false, B, w, as_stream(stream), q8);
 }
 

@@ -164,7 +164,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, int m, int n0, int
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       float v[32];
-      ld_acc(taddr + 32 * c, v);
+      ld_acc_s<F8>(taddr + 32 * c, v, sa, e.b_scale + n0 + 32 * c);
       if (active) {
         float xv[32];
         const size_t off = (size_t)m * N + n0 + 32 * c;
@@ -480,6 +480,8 @@ cudaError_t launch_gemm_e4m3(int epi, int M, int N, int K, const void* A, const 
   switch (epi) {
     case EPI_QKV: return run<EPI_QKV, 256, true>(M, N, K, A, Bm, e, st);
     case EPI_SWIGLU: return run<EPI_SWIGLU, 256, true>(M, N, K, A, Bm, e, st);
+    case EPI_RESID: return run<EPI_RESID, 256, true>(M, N, K, A, Bm, e, st);
+    case EPI_RESID_F32: return run<EPI_RESID_F32, 256, true>(M, N, K, A, Bm, e, st);
     default: return cudaErrorInvalidValue;
   }
 }

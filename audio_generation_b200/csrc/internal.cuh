@@ -204,7 +204,8 @@ cudaError_t launch_gemm(int epi, int M, int N, int K, const void* A, const void*
                         const GemmEpiArgs& e, cudaStream_t st);
 
 // The same product on e4m3 codes (A [M, K], B [N, K] bytes) with
-// C[m, n] = a_scale[m] * b_scale[n] * (A . B^T)[m, n]; EPI_QKV or EPI_SWIGLU.
+// C[m, n] = a_scale[m] * b_scale[n] * (A . B^T)[m, n]; EPI_QKV, EPI_SWIGLU,
+// EPI_RESID or EPI_RESID_F32 (N % 256 == 0, K % 128 == 0).
 cudaError_t launch_gemm_e4m3(int epi, int M, int N, int K, const void* A, const void* Bm,
                              const GemmEpiArgs& e, cudaStream_t st);
 

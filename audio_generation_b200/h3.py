@@ -68,7 +68,8 @@ class h3_io_weights(ctypes.Structure):
 
 class h3_block_weights_e4m3(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
-        "w_qkv_codes", "w_qkv_scales", "w13_codes", "w13_scales")]
+        "w_qkv_codes", "w_qkv_scales", "w13_codes", "w13_scales", "w_o_codes", "w_o_scales",
+        "w2_codes", "w2_scales")]
 
 
 H3_MAX_RANKS = 8
@@ -120,6 +121,10 @@ _SIGNATURES = {
     "h3_qkv_rope_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                               _vp, _vp, _vp, _vp]),
     "h3_ffn_up_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "h3_out_residual_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp, _vp,
+                                  _vp, _vp, _vp]),
+    "h3_ffn_down_residual_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp,
+                                       _vp, _vp, _vp, _vp]),
     "h3_workspace_size_e4m3": (_sz, [ctypes.POINTER(h3_dims), _i, _i]),
     "h3_block_forward_e4m3": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights),
                                    ctypes.POINTER(h3_block_weights_e4m3), _vp, _vp, _vp, _i, _vp,
@@ -464,9 +469,27 @@ def h3_ffn_up_e4m3(dims: h3_dims, layout: Layout, B: int, h2_codes, h2_scales, w
                                 _stream(stream)), "h3_ffn_up_e4m3")
 
 
-def make_block_weights_e4m3(w_qkv_codes, w_qkv_scales, w13_codes, w13_scales):
+def make_block_weights_e4m3(w_qkv_codes, w_qkv_scales, w13_codes, w13_scales, w_o_codes=None,
+                            w_o_scales=None, w2_codes=None, w2_scales=None):
     return h3_block_weights_e4m3(*[_ptr(t) for t in (w_qkv_codes, w_qkv_scales, w13_codes,
-                                                     w13_scales)])
+                                                     w13_scales, w_o_codes, w_o_scales, w2_codes,
+                                                     w2_scales)])
+
+
+def h3_out_residual_e4m3(dims: h3_dims, layout: Layout, B: int, o_codes, o_scales, w_codes,
+                         w_scales, ada_table, tmod, x, stream=None) -> None:
+    _check(lib().h3_out_residual_e4m3(ctypes.byref(dims), layout.handle, B, _ptr(o_codes),
+                                      _ptr(o_scales), _ptr(w_codes), _ptr(w_scales),
+                                      _ptr(ada_table), _ptr(tmod), _ptr(x), _stream(stream)),
+           "h3_out_residual_e4m3")
+
+
+def h3_ffn_down_residual_e4m3(dims: h3_dims, layout: Layout, B: int, g_codes, g_scales, w_codes,
+                              w_scales, ada_table, tmod, x, stream=None) -> None:
+    _check(lib().h3_ffn_down_residual_e4m3(ctypes.byref(dims), layout.handle, B, _ptr(g_codes),
+                                           _ptr(g_scales), _ptr(w_codes), _ptr(w_scales),
+                                           _ptr(ada_table), _ptr(tmod), _ptr(x), _stream(stream)),
+           "h3_ffn_down_residual_e4m3")
 
 
 def h3_workspace_size_e4m3(dims: h3_dims, B: int, S: int) -> int:

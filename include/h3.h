@@ -342,12 +342,21 @@ H3_API h3_status h3_quantize_e4m3_rows(const void* w, int rows, int K, void* cod
                                        h3_stream_t stream);
 
 /* The 8-bit operands of one block (DEVICE pointers, from h3_quantize_e4m3_rows
- * applied to the block's w_qkv [3*NH*D, H] and w13 [2F, H]). */
+ * applied to the block's w_qkv [3*NH*D, H] and w13 [2F, H], and optionally to
+ * w_o [H, NH*D] and w2 [H, F]). With w_o_codes (w2_codes) null the output
+ * projection (FFN down projection) stays bf16; with them set, its input rows
+ * (o, g: bf16 as stored) are quantized per row first, one scale per row as for
+ * h ("Sampler en DiT controls": an 8-bit FC2 with one activation scale per
+ * row). The 8-bit O and W2 GEMMs need hidden % 256 == 0. */
 typedef struct {
   const void* w_qkv_codes;
   const float* w_qkv_scales;
   const void* w13_codes;
   const float* w13_scales;
+  const void* w_o_codes;   /* may be null */
+  const float* w_o_scales;
+  const void* w2_codes;    /* may be null */
+  const float* w2_scales;
 } h3_block_weights_e4m3;
 
 /* The steps of the 8-bit block, each as in the bf16 step of the same name.
@@ -377,12 +386,28 @@ H3_API h3_status h3_ffn_up_e4m3(const h3_dims* dims, h3_layout_t layout, int B,
                                 const void* h2_codes, const float* h2_scales, const void* w_codes,
                                 const float* w_scales, void* g, h3_stream_t stream);
 
+/* h3_out_residual and h3_ffn_down_residual on 8-bit operands: input codes
+ * [B*S, K] with per-row scales [B*S] (K = heads*128, resp. ffn), weight codes
+ * [H, K] with per-row scales [H]; the gated residual as in the bf16 steps.
+ * hidden % 256 == 0. */
+H3_API h3_status h3_out_residual_e4m3(const h3_dims* dims, h3_layout_t layout, int B,
+                                      const void* o_codes, const float* o_scales,
+                                      const void* w_codes, const float* w_scales,
+                                      const float* ada_table, const float* tmod, void* x,
+                                      h3_stream_t stream);
+H3_API h3_status h3_ffn_down_residual_e4m3(const h3_dims* dims, h3_layout_t layout, int B,
+                                           const void* g_codes, const float* g_scales,
+                                           const void* w_codes, const float* w_scales,
+                                           const float* ada_table, const float* tmod, void* x,
+                                           h3_stream_t stream);
+
 /* Workspace bytes of h3_block_forward_e4m3: h3_workspace_size plus the codes
- * [B*S, H] and scales [B*S] of the activation rows. */
+ * [B*S, max(H, heads*128, ffn)] and scales [B*S] of the activation rows. */
 H3_API size_t h3_workspace_size_e4m3(const h3_dims* dims, int B, int S);
 
-/* h3_block_forward with the QKV and W1 || W3 GEMMs on e4m3 operands (the bf16
- * w_qkv and w13 of `weights` are not read). hidden % 128 == 0. */
+/* h3_block_forward with the QKV and W1 || W3 GEMMs (and, where w8 has them, the
+ * O and W2 GEMMs) on e4m3 operands; the bf16 weights they replace are not
+ * read. hidden % 128 == 0 (% 256 with O or W2 in 8 bits). */
 H3_API h3_status h3_block_forward_e4m3(const h3_dims* dims, const h3_block_weights* weights,
                                        const h3_block_weights_e4m3* w8, h3_layout_t layout,
                                        const float* tmod, void* x, int B, void* ws,

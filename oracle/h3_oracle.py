@@ -238,8 +238,14 @@ def attention(q: np.ndarray, doc_q: np.ndarray, k: np.ndarray, v: np.ndarray,
 
 def out_project_residual(x: np.ndarray, o: np.ndarray, gate: np.ndarray, w_o: np.ndarray,
                          emulate: bool = False) -> np.ndarray:
-    """x1 = x + gate * (o W_o^T)."""
-    return _store(x + gate * (o @ bf16_to_f64(w_o).T), emulate)
+    """x1 = x + gate * (o W_o^T); w_o as bf16 bits."""
+    return out_project_residual_values(x, o, gate, bf16_to_f64(w_o), emulate)
+
+
+def out_project_residual_values(x: np.ndarray, o: np.ndarray, gate: np.ndarray, w_o: np.ndarray,
+                                emulate: bool = False) -> np.ndarray:
+    """out_project_residual with W_o [H, NH D] given as values."""
+    return _store(x + gate * (o @ np.asarray(w_o, F).T), emulate)
 
 
 def ffn_gate(h2: np.ndarray, w13: np.ndarray, ffn: int, emulate: bool = False) -> np.ndarray:
@@ -255,8 +261,14 @@ def ffn_gate_values(h2: np.ndarray, w13: np.ndarray, ffn: int, emulate: bool = F
 
 def ffn_down_residual(x1: np.ndarray, g: np.ndarray, gate: np.ndarray, w2: np.ndarray,
                       emulate: bool = False) -> np.ndarray:
-    """x2 = x1 + gate * (g W2^T)."""
-    return _store(x1 + gate * (g @ bf16_to_f64(w2).T), emulate)
+    """x2 = x1 + gate * (g W2^T); w2 as bf16 bits."""
+    return ffn_down_residual_values(x1, g, gate, bf16_to_f64(w2), emulate)
+
+
+def ffn_down_residual_values(x1: np.ndarray, g: np.ndarray, gate: np.ndarray, w2: np.ndarray,
+                             emulate: bool = False) -> np.ndarray:
+    """ffn_down_residual with W2 [H, F] given as values."""
+    return _store(x1 + gate * (g @ np.asarray(w2, F).T), emulate)
 
 
 # --------------------------------------------------------------------------
@@ -561,11 +573,13 @@ def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 
 
 def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
-                      emulate: bool = False) -> np.ndarray:
+                      emulate: bool = False, out_down: bool = False) -> np.ndarray:
     """The block with its QKV and W1 || W3 GEMMs on e4m3 inputs: the norm outputs
     h and h2 quantized per row (their values held in float32, as the device
     holds them) and the bf16 weights per output channel; everything else as in
-    block_forward. (B = 1 or more; padding rows unchanged.)
+    block_forward. (B = 1 or more; padding rows unchanged.) With ``out_down``
+    the O and W2 GEMMs take e4m3 inputs too: o and g quantized per row from
+    their values as stored, W_o and W2 per output channel.
 
     ``emulate`` rounds to bf16 where the device stores bf16 in this block (q, k, v
     after RoPE, P, o, x1, g, x2; h and h2 go from fp32 straight to codes). A
@@ -574,7 +588,7 @@ def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
     the norm2 input x1 has to be the bf16 value the device stored."""
     import copy
     wq = copy.copy(w)
-    for name in ("w_qkv", "w13"):
+    for name in ("w_qkv", "w13") + (("w_o", "w2") if out_down else ()):
         wf = bf16_to_f64(getattr(w, name)).astype(np.float32)
         codes, sc = quantize_rows_e4m3(wf)
         setattr(wq, name, dequantize_rows(codes, sc))
@@ -590,11 +604,19 @@ def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
         hq = dequantize_rows(*quantize_rows_e4m3(h))
         q, k, v = qkv_project_values(hq, layout.pos, wq.w_qkv, w.q_norm, w.k_norm, dims, emulate)
         o = attention(q, pad, k, v, pad, emulate)
-        x1 = out_project_residual(x[b], o, m[:, 2], w.w_o, emulate)
+        if out_down:
+            x1 = out_project_residual_values(x[b], dequantize_rows(*quantize_rows_e4m3(o)),
+                                             m[:, 2], wq.w_o, emulate)
+        else:
+            x1 = out_project_residual(x[b], o, m[:, 2], w.w_o, emulate)
         h2 = norm_modulate(x1, m[:, 3], m[:, 4], dims.norm_eps)
         h2q = dequantize_rows(*quantize_rows_e4m3(h2))
         g = ffn_gate_values(h2q, wq.w13, dims.ffn, emulate)
-        y = ffn_down_residual(x1, g, m[:, 5], w.w2, emulate)
+        if out_down:
+            y = ffn_down_residual_values(x1, dequantize_rows(*quantize_rows_e4m3(g)), m[:, 5],
+                                         wq.w2, emulate)
+        else:
+            y = ffn_down_residual(x1, g, m[:, 5], w.w2, emulate)
         out[b] = np.where(pad[:, None], x[b], y)
     return out
 

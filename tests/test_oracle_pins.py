@@ -1078,3 +1078,9 @@ def test_fp8_block_is_close_to_the_block_and_keeps_padding():
     d, d8 = y[0, ~pad] - x[0, ~pad], y8[0, ~pad] - x[0, ~pad]
     r = _rel(d8, d)
     assert 1e-3 < r < 0.08, r
+    # with the O and W2 inputs in 8 bits too: still near the block, a little
+    # further from it, padding unchanged
+    y8a = O.block_forward_fp8(x, w, L, tmod, SMALL, out_down=True)
+    np.testing.assert_array_equal(y8a[0, pad], x[0, pad])
+    ra = _rel(y8a[0, ~pad] - x[0, ~pad], d)
+    assert r < ra < 0.1, (r, ra)
