@@ -625,17 +625,23 @@ STACK_WORKLOAD = ("full-width MiniMax-H3 50-block stack forward, S=16384 packed 
 
 
 def run_stack(args):
-    """--stack: the 50-block stack forward on one GPU, one JSON line."""
-    print(json.dumps(stack_measure(args.steps, args.warmup)))
+    """--stack: the 50-block stack forward on one GPU, one JSON line; with
+    --reduced also the token-reduced stack (blocks [3, 39) on the reduced
+    sequence, the page's schedule)."""
+    print(json.dumps(stack_measure(args.steps, args.warmup,
+                                   (3, 39) if args.reduced else None)))
     return 0
 
 
-def stack_measure(steps, warmup):
+def stack_measure(steps, warmup, reduce_blocks=None):
     """The 50-block stack forward on one GPU (layout prepared once, the
     per-forward prologue for the two timesteps, then the stack with the valid rows
     gathered into an fp32 stream and scattered back): forward time, valid rows/s
     and TFLOP/s (algorithmic flops of 50 blocks over the valid rows and the valid
-    document)."""
+    document). With ``reduce_blocks = (r0, r1)`` the stack runs blocks [r0, r1)
+    on the token-reduced sequence (h3_stack_forward_reduced: pairs of adjacent
+    target-video rows, the video rows of frames t >= 1, merged), and the line
+    reports the plain stack's time beside it."""
     import torch
     from audio_generation_b200 import h3
 
@@ -687,22 +693,45 @@ def stack_measure(steps, warmup):
         h3.h3_timestep_modulation(d, L.n_t, t_dev, w1, w2p, wp, tmod, tws, tws_b, stream)
         h3.h3_stack_forward(d, cws, layout, tmod, x, 1, ws, ws_b, stream)
 
-    for _ in range(warmup):
-        forward()
-    torch.cuda.synchronize(device)
     gpu_id = torch.cuda.get_device_properties(device).uuid
     gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(gpu_id) as clk:
-        time.sleep(0.3)
-        e0.record(stream)
-        for _ in range(steps):
-            forward()
-        e1.record(stream)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
         torch.cuda.synchronize(device)
-    if h3.h3_layout_error(layout) != h3.H3_OK:
-        raise RuntimeError("device error word set during the stack run")
-    ms = e0.elapsed_time(e1) / steps
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(gpu_id) as clk:
+            time.sleep(0.3)
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+        if h3.h3_layout_error(layout) != h3.H3_OK:
+            raise RuntimeError("device error word set during the stack run")
+        return e0.elapsed_time(e1) / steps, clk
+
+    reduced = None
+    if reduce_blocks is not None:
+        r0, r1 = reduce_blocks
+        target = ((L.tags == 0) & (L.pos[:, 0] >= 1)).astype(np.int32)
+        red = h3.h3_layout_reduce(d, layout, to_dev_i32(target))
+        rws_b = h3.h3_stack_reduced_workspace_size(d, layout, red, 1)
+        rws = torch.empty(rws_b, dtype=torch.uint8, device=device)
+
+        def forward_reduced():
+            x.copy_(x0, non_blocking=True)
+            h3.h3_timestep_modulation(d, L.n_t, t_dev, w1, w2p, wp, tmod, tws, tws_b, stream)
+            h3.h3_stack_forward_reduced(d, cws, layout, red, r0, r1, tmod, x, 1, rws, rws_b,
+                                        stream)
+
+        ms_red, clk_red = timed(forward_reduced)
+        reduced = {"ms_per_step": ms_red, "value": V / (ms_red * 1e-3), "r0": r0, "r1": r1,
+                   "target_rows": int(target.sum()), "clocks": clk_red.summary()}
+        red.close()
+        del rws
+    ms, clk = timed(forward)
     flops = STACK_BLOCKS * block_flops(dims, V)
     peaks = load_peaks()
     tflops = flops / (ms * 1e-3) / 1e12
@@ -717,6 +746,9 @@ def stack_measure(steps, warmup):
         "frac_of_burst_peak": tflops / peaks["bf16_tflops"], "clocks": clk.summary(),
         "gpu_launches": steps * (4 + 2 + 7 * STACK_BLOCKS),  # prologue, gather / scatter, blocks
     }
+    if reduced is not None:
+        reduced["speedup_vs_full_stack"] = ms / reduced["ms_per_step"]
+        line["token_reduced"] = reduced
     layout.close()
     return line
 
@@ -896,6 +928,24 @@ def run_forward(args):
     if h3.h3_layout_error(layout) != h3.H3_OK:
         raise RuntimeError("device error word set during the forward run")
     ms = e0.elapsed_time(e1) / args.steps
+    # core residual reuse: one forward that stores the stack's change, then
+    # forwards that reuse it (the refiner and the 50 blocks skipped)
+    core = torch.empty((1, V, dims.hidden), dtype=torch.float32, device=device)
+    h3.h3_forward(d, io, iw, refiner, blocks, layout, ts, 1, v_d, a_d, t_d, vo, ao, ws, ws_b,
+                  stream, core, h3.H3_CORE_STORE)
+    for _ in range(args.warmup):
+        h3.h3_forward(d, io, iw, refiner, blocks, layout, ts, 1, v_d, a_d, t_d, vo, ao, ws, ws_b,
+                      stream, core, h3.H3_CORE_REUSE)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(args.steps):
+        h3.h3_forward(d, io, iw, refiner, blocks, layout, ts, 1, v_d, a_d, t_d, vo, ao, ws, ws_b,
+                      stream, core, h3.H3_CORE_REUSE)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    if h3.h3_layout_error(layout) != h3.H3_OK:
+        raise RuntimeError("device error word set during the core-reuse run")
+    ms_reuse = e0.elapsed_time(e1) / args.steps
     H = dims.hidden
     flops = (STACK_BLOCKS * block_flops(dims, V) + 2 * block_flops(dims, nt_rows)
              + 2.0 * nt_rows * dims.text_dim * H
@@ -912,6 +962,9 @@ def run_forward(args):
                    "refiner_blocks": len(refiner), "text_rows": nt_rows, "n_t": int(L.n_t)},
         "tflops": tflops, "frac_of_sustained_peak": tflops / peaks["bf16_tflops_sustained"],
         "frac_of_burst_peak": tflops / peaks["bf16_tflops"], "clocks": clk.summary(),
+        "core_reuse": {"ms_per_step": ms_reuse,
+                       "note": "H3_CORE_REUSE forward: projections, norm_out and heads over the "
+                               "stored core residual (refiner and stack skipped)"},
     }
     print(json.dumps(line))
     layout.close()
@@ -933,6 +986,8 @@ def main(argv=None):
                     help="skip the 50-block stack measurement added to the block line")
     ap.add_argument("--no-masked", action="store_true",
                     help="skip the masked-attention measurement on the padded layout")
+    ap.add_argument("--reduced", action="store_true",
+                    help="with --stack: also time the token-reduced stack")
     ap.add_argument("--stack", action="store_true",
                     help="time the 50-block stack forward instead (one GPU, own JSON line)")
     ap.add_argument("--attention-only", action="store_true",
