@@ -981,6 +981,29 @@ size_t h3_workspace_size_e4m3(const h3_dims* dims, int B, int S) {
 
 namespace {
 
+h3_status check_w8(const h3_dims* dims, const h3_block_weights_e4m3* w8) {
+  if (!w8 || !w8->w_qkv_codes || !w8->w_qkv_scales || !w8->w13_codes || !w8->w13_scales)
+    return H3_ERR_ARG;
+  if ((w8->w_o_codes && !w8->w_o_scales) || (w8->w2_codes && !w8->w2_scales)) return H3_ERR_ARG;
+  if (!aligned16(w8->w_qkv_codes) || !aligned16(w8->w_qkv_scales) || !aligned16(w8->w13_codes) ||
+      !aligned16(w8->w13_scales) || !aligned16(w8->w_o_codes) || !aligned16(w8->w_o_scales) ||
+      !aligned16(w8->w2_codes) || !aligned16(w8->w2_scales))
+    return H3_ERR_ALIGN;
+  if (dims->hidden % 128 != 0) return H3_ERR_SHAPE;
+  if ((w8->w_o_codes || w8->w2_codes) && dims->hidden % 256 != 0) return H3_ERR_SHAPE;
+  return H3_OK;
+}
+
+E4m3Operands e4m3_operands(const h3_dims& d, int B, int S, void* ws, size_t base,
+                           const h3_block_weights_e4m3* w8) {
+  E4m3Operands q8;
+  q8.w = w8;
+  q8.codes = static_cast<uint8_t*>(ws) + base;
+  q8.scales = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + base +
+                                       align256((size_t)B * S * e4m3_row_bytes(d)));
+  return q8;
+}
+
 h3_status resid_e4m3(const h3_dims* dims, h3_layout_t L, int B, int K, int gate_chunk,
                      const void* a_codes, const float* a_scales, const void* w_codes,
                      const float* w_scales, const float* ada_table, const float* tmod, void* x,
@@ -1038,25 +1061,41 @@ h3_status h3_block_forward_e4m3(const h3_dims* dims, const h3_block_weights* wei
   if (!L || B < 0 || !tmod || !x || !ws || !w8) return H3_ERR_ARG;
   H3_TRY(check_batch(L, B));
   H3_TRY(check_weights(weights));
-  if (!w8->w_qkv_codes || !w8->w_qkv_scales || !w8->w13_codes || !w8->w13_scales)
-    return H3_ERR_ARG;
-  if ((w8->w_o_codes && !w8->w_o_scales) || (w8->w2_codes && !w8->w2_scales)) return H3_ERR_ARG;
-  if (!aligned16(w8->w_qkv_codes) || !aligned16(w8->w_qkv_scales) || !aligned16(w8->w13_codes) ||
-      !aligned16(w8->w13_scales) || !aligned16(w8->w_o_codes) || !aligned16(w8->w_o_scales) ||
-      !aligned16(w8->w2_codes) || !aligned16(w8->w2_scales) || !aligned16(tmod) ||
-      !aligned16(x) || !aligned16(ws))
-    return H3_ERR_ALIGN;
-  if (dims->hidden % 128 != 0) return H3_ERR_SHAPE;
-  if ((w8->w_o_codes || w8->w2_codes) && dims->hidden % 256 != 0) return H3_ERR_SHAPE;
+  H3_TRY(check_w8(dims, w8));
+  if (!aligned16(tmod) || !aligned16(x) || !aligned16(ws)) return H3_ERR_ALIGN;
   if (ws_bytes < h3_workspace_size_e4m3(dims, B, L->S)) return H3_ERR_WORKSPACE;
   Workspace w;
   const size_t base = ws_parts(*dims, B, L->S, &w, ws);
-  E4m3Operands q8;
-  q8.w = w8;
-  q8.codes = static_cast<uint8_t*>(ws) + base;
-  q8.scales = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + base +
-                                       align256((size_t)B * L->S * e4m3_row_bytes(*dims)));
+  const E4m3Operands q8 = e4m3_operands(*dims, B, L->S, ws, base, w8);
   return run_block(*dims, *weights, L->view(), tmod, x, false, B, w, as_stream(stream), q8);
+}
+
+h3_status h3_stack_forward_e4m3(const h3_dims* dims, const h3_block_weights* weights,
+                                const h3_block_weights_e4m3* w8, int n_blocks, h3_layout_t L,
+                                const float* tmod, void* x, int B, void* ws, size_t ws_bytes,
+                                h3_stream_t stream) {
+  H3_TRY(check_dims(dims));
+  if (!L || B < 0 || n_blocks < 0 || !tmod || !x || !ws || (n_blocks > 0 && (!weights || !w8)))
+    return H3_ERR_ARG;
+  H3_TRY(check_batch(L, B));
+  for (int i = 0; i < n_blocks; ++i) {
+    H3_TRY(check_weights(&weights[i]));
+    H3_TRY(check_w8(dims, &w8[i]));
+  }
+  if (!aligned16(tmod) || !aligned16(x) || !aligned16(ws)) return H3_ERR_ALIGN;
+  if (ws_bytes < h3_workspace_size_e4m3(dims, B, L->S)) return H3_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  Workspace w;
+  const size_t base = ws_parts(*dims, B, L->S, &w, ws);
+  // as h3_stack_forward: the valid rows in an fp32 residual stream
+  const int V = L->n_valid;
+  H3_CUDA(launch_permute_rows_convert(B, V, L->S, dims->hidden, L->perm, x, w.xc, true, st));
+  for (int i = 0; i < n_blocks; ++i) {
+    const E4m3Operands q8 = e4m3_operands(*dims, B, L->S, ws, base, &w8[i]);
+    H3_TRY(run_block(*dims, weights[i], L->compact_view(), tmod, w.xc, true, B, w, st, q8));
+  }
+  H3_CUDA(launch_permute_rows_convert(B, V, L->S, dims->hidden, L->perm, w.xc, x, false, st));
+  return H3_OK;
 }
 
 }  // extern "C"

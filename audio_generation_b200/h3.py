@@ -126,6 +126,9 @@ _SIGNATURES = {
     "h3_ffn_down_residual_e4m3": (_i, [ctypes.POINTER(h3_dims), _vp, _i, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _vp, _vp]),
     "h3_workspace_size_e4m3": (_sz, [ctypes.POINTER(h3_dims), _i, _i]),
+    "h3_stack_forward_e4m3": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights),
+                                   ctypes.POINTER(h3_block_weights_e4m3), _i, _vp, _vp, _vp, _i,
+                                   _vp, _sz, _vp]),
     "h3_block_forward_e4m3": (_i, [ctypes.POINTER(h3_dims), ctypes.POINTER(h3_block_weights),
                                    ctypes.POINTER(h3_block_weights_e4m3), _vp, _vp, _vp, _i, _vp,
                                    _sz, _vp]),
@@ -474,6 +477,19 @@ def make_block_weights_e4m3(w_qkv_codes, w_qkv_scales, w13_codes, w13_scales, w_
     return h3_block_weights_e4m3(*[_ptr(t) for t in (w_qkv_codes, w_qkv_scales, w13_codes,
                                                      w13_scales, w_o_codes, w_o_scales, w2_codes,
                                                      w2_scales)])
+
+
+def h3_stack_forward_e4m3(dims: h3_dims, weights: Sequence[h3_block_weights],
+                          w8: Sequence[h3_block_weights_e4m3], layout: Layout, tmod, x, B: int,
+                          ws, ws_bytes: int, stream=None) -> None:
+    if len(weights) != len(w8):
+        raise ValueError("one set of 8-bit operands per block")
+    n = len(weights)
+    arr = (h3_block_weights * max(1, n))(*weights)
+    arr8 = (h3_block_weights_e4m3 * max(1, n))(*w8)
+    _check(lib().h3_stack_forward_e4m3(ctypes.byref(dims), arr, arr8, n, layout.handle, _ptr(tmod),
+                                       _ptr(x), B, _ptr(ws), ws_bytes, _stream(stream)),
+           "h3_stack_forward_e4m3")
 
 
 def h3_out_residual_e4m3(dims: h3_dims, layout: Layout, B: int, o_codes, o_scales, w_codes,

@@ -629,11 +629,11 @@ def run_stack(args):
     --reduced also the token-reduced stack (blocks [3, 39) on the reduced
     sequence, the page's schedule)."""
     print(json.dumps(stack_measure(args.steps, args.warmup,
-                                   (3, 39) if args.reduced else None)))
+                                   (3, 39) if args.reduced else None, e4m3=args.e4m3)))
     return 0
 
 
-def stack_measure(steps, warmup, reduce_blocks=None):
+def stack_measure(steps, warmup, reduce_blocks=None, e4m3=False):
     """The 50-block stack forward on one GPU (layout prepared once, the
     per-forward prologue for the two timesteps, then the stack with the valid rows
     gathered into an fp32 stream and scattered back): forward time, valid rows/s
@@ -641,7 +641,9 @@ def stack_measure(steps, warmup, reduce_blocks=None):
     document). With ``reduce_blocks = (r0, r1)`` the stack runs blocks [r0, r1)
     on the token-reduced sequence (h3_stack_forward_reduced: pairs of adjacent
     target-video rows, the video rows of frames t >= 1, merged), and the line
-    reports the plain stack's time beside it."""
+    reports the plain stack's time beside it. With ``e4m3`` every block runs its
+    four GEMMs on e4m3 operands (h3_stack_forward_e4m3; weights quantized once,
+    before timing)."""
     import torch
     from audio_generation_b200 import h3
 
@@ -662,7 +664,7 @@ def stack_measure(steps, warmup, reduce_blocks=None):
     def to_dev_i32(a):
         return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
 
-    keep, cws = [], []
+    keep, cws, w8s = [], [], []
     for i in range(STACK_BLOCKS):
         w = block_weights(dims, STACK_CFG, i)
         t = {k: to_dev_bits(getattr(w, k)) for k in ("w_qkv", "q_norm", "k_norm", "w_o", "w13",
@@ -671,6 +673,15 @@ def stack_measure(steps, warmup, reduce_blocks=None):
         keep.append(t)
         cws.append(h3.make_block_weights(t["w_qkv"], t["q_norm"], t["k_norm"], t["w_o"],
                                          t["w13"], t["w2"], t["ada_table"]))
+        if e4m3:
+            q = {}
+            for name in ("w_qkv", "w13", "w_o", "w2"):
+                rows, K = getattr(w, name).shape
+                q[name] = (torch.empty((rows, K), dtype=torch.uint8, device=device),
+                           torch.empty(rows, dtype=torch.float32, device=device))
+                h3.h3_quantize_e4m3_rows(t[name], rows, K, q[name][0], q[name][1])
+            t["q8"] = q
+            w8s.append(h3.make_block_weights_e4m3(*q["w_qkv"], *q["w13"], *q["w_o"], *q["w2"]))
     pw = prologue_weights(dims, STACK_CFG)
     pos, tags, tidx = to_dev_f32(L.pos), to_dev_i32(L.tags), to_dev_i32(L.t_idx)
     vi, ai, ti = to_dev_i32(L.video_idx), to_dev_i32(L.audio_idx), to_dev_i32(L.text_idx)
@@ -684,14 +695,17 @@ def stack_measure(steps, warmup, reduce_blocks=None):
         torch.bfloat16)
     x0 = x_host.to(device)
     x = torch.empty_like(x0)
-    ws_b = h3.h3_workspace_size(d, 1, S)
+    ws_b = (h3.h3_workspace_size_e4m3 if e4m3 else h3.h3_workspace_size)(d, 1, S)
     ws = torch.empty(ws_b, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
     def forward():
         x.copy_(x0, non_blocking=True)
         h3.h3_timestep_modulation(d, L.n_t, t_dev, w1, w2p, wp, tmod, tws, tws_b, stream)
-        h3.h3_stack_forward(d, cws, layout, tmod, x, 1, ws, ws_b, stream)
+        if e4m3:
+            h3.h3_stack_forward_e4m3(d, cws, w8s, layout, tmod, x, 1, ws, ws_b, stream)
+        else:
+            h3.h3_stack_forward(d, cws, layout, tmod, x, 1, ws, ws_b, stream)
 
     gpu_id = torch.cuda.get_device_properties(device).uuid
     gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
@@ -736,16 +750,23 @@ def stack_measure(steps, warmup, reduce_blocks=None):
     peaks = load_peaks()
     tflops = flops / (ms * 1e-3) / 1e12
     line = {
-        "metric": "valid packed rows/s per 50-block stack forward (bf16, 1xB200)",
+        "metric": "valid packed rows/s per 50-block stack forward (%s, 1xB200)" % (
+            "e4m3 GEMM operands" if e4m3 else "bf16"),
         "value": V / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": steps,
-        "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16",
+        "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
+        "dtype": "e4m3 (QKV, O, W1||W3, W2) + bf16 (attention)" if e4m3 else "bf16",
         "data": "synthetic (seeded random-init weights and activations)",
         "config": {"workload": STACK_WORKLOAD, "S": S, "valid_rows": V, "blocks": STACK_BLOCKS,
                    "n_t": int(L.n_t)},
-        "tflops": tflops, "frac_of_sustained_peak": tflops / peaks["bf16_tflops_sustained"],
-        "frac_of_burst_peak": tflops / peaks["bf16_tflops"], "clocks": clk.summary(),
-        "gpu_launches": steps * (4 + 2 + 7 * STACK_BLOCKS),  # prologue, gather / scatter, blocks
+        "tflops": tflops, "clocks": clk.summary(),
+        # prologue, gather / scatter, blocks (two row-quantizing passes more in 8 bits)
+        "gpu_launches": steps * (4 + 2 + (9 if e4m3 else 7) * STACK_BLOCKS),
     }
+    # fractions of the bf16 peaks (an 8-bit stack's flops are counted as the
+    # bf16 stack's, so its fractions can exceed 1)
+    pre = "frac_of_bf16_" if e4m3 else "frac_of_"
+    line[pre + "sustained_peak"] = tflops / peaks["bf16_tflops_sustained"]
+    line[pre + "burst_peak"] = tflops / peaks["bf16_tflops"]
     if reduced is not None:
         reduced["speedup_vs_full_stack"] = ms / reduced["ms_per_step"]
         line["token_reduced"] = reduced

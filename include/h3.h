@@ -413,6 +413,14 @@ H3_API h3_status h3_block_forward_e4m3(const h3_dims* dims, const h3_block_weigh
                                        const float* tmod, void* x, int B, void* ws,
                                        size_t ws_bytes, h3_stream_t stream);
 
+/* h3_stack_forward with every block on its 8-bit operands w8[i] (as
+ * h3_block_forward_e4m3), over the stack's fp32 residual stream. ws:
+ * h3_workspace_size_e4m3(dims, B, S) bytes. */
+H3_API h3_status h3_stack_forward_e4m3(const h3_dims* dims, const h3_block_weights* weights,
+                                       const h3_block_weights_e4m3* w8, int n_blocks,
+                                       h3_layout_t layout, const float* tmod, void* x, int B,
+                                       void* ws, size_t ws_bytes, h3_stream_t stream);
+
 /* ---- token reduction in the middle blocks ---- */
 
 /* Build the token-reduced layout of `full` ("MiniMax H3 Inference Engine voor

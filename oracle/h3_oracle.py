@@ -573,7 +573,8 @@ def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 
 
 def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
-                      emulate: bool = False, out_down: bool = False) -> np.ndarray:
+                      emulate: bool = False, out_down: bool = False,
+                      stream_f32: bool = False) -> np.ndarray:
     """The block with its QKV and W1 || W3 GEMMs on e4m3 inputs: the norm outputs
     h and h2 quantized per row (their values held in float32, as the device
     holds them) and the bf16 weights per output channel; everything else as in
@@ -585,7 +586,9 @@ def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
     after RoPE, P, o, x1, g, x2; h and h2 go from fp32 straight to codes). A
     code is an integer that floating point decides: compared with the device,
     the reference must take that decision from the values the device holds, so
-    the norm2 input x1 has to be the bf16 value the device stored."""
+    the norm2 input x1 has to be the bf16 value the device stored. With
+    ``stream_f32`` (and ``emulate``) x1 and the output are held in fp32 instead,
+    as a stack's residual stream holds them."""
     import copy
     wq = copy.copy(w)
     for name in ("w_qkv", "w13") + (("w_o", "w2") if out_down else ()):
@@ -606,17 +609,19 @@ def block_forward_fp8(x: np.ndarray, w, layout, tmod: np.ndarray, dims,
         o = attention(q, pad, k, v, pad, emulate)
         if out_down:
             x1 = out_project_residual_values(x[b], dequantize_rows(*quantize_rows_e4m3(o)),
-                                             m[:, 2], wq.w_o, emulate)
+                                             m[:, 2], wq.w_o)
         else:
-            x1 = out_project_residual(x[b], o, m[:, 2], w.w_o, emulate)
+            x1 = out_project_residual(x[b], o, m[:, 2], w.w_o)
+        x1 = _stream(x1, emulate, stream_f32)
         h2 = norm_modulate(x1, m[:, 3], m[:, 4], dims.norm_eps)
         h2q = dequantize_rows(*quantize_rows_e4m3(h2))
         g = ffn_gate_values(h2q, wq.w13, dims.ffn, emulate)
         if out_down:
             y = ffn_down_residual_values(x1, dequantize_rows(*quantize_rows_e4m3(g)), m[:, 5],
-                                         wq.w2, emulate)
+                                         wq.w2)
         else:
-            y = ffn_down_residual(x1, g, m[:, 5], w.w2, emulate)
+            y = ffn_down_residual(x1, g, m[:, 5], w.w2)
+        y = _stream(y, emulate, stream_f32)
         out[b] = np.where(pad[:, None], x[b], y)
     return out
 

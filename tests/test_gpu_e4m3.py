@@ -342,3 +342,72 @@ def test_e4m3_block_full_width(out_down):
     assert_close(got[~pad] - x0[~pad], ref[~pad] - x0[~pad], what="full-width e4m3 update",
                  rel=REL_L2 + sp.upd, mabs=np.inf)
     np.testing.assert_array_equal(got[pad], x0[pad])
+
+
+def _stack_refs(x0, ws_host, L, tm, dims, out_down):
+    """The oracle's 8-bit blocks in sequence over an fp32 stream, rounded to bf16
+    once at the end (as the stack scatters its rows back): the bf16-storage
+    reading and the float64 one."""
+    refs = []
+    for emulate in (True, False):
+        y = x0[None]
+        for w in ws_host:
+            y = O.block_forward_fp8(y, w, L, tm, dims, emulate=emulate, out_down=out_down,
+                                    stream_f32=True)
+        refs.append(O.round_bf16(y[0]) if emulate else y[0])
+    return refs
+
+
+def gpu_stack_e4m3(dims, L, ws_host, tmod, xb, out_down):
+    dl = DevLayout(dims, L)
+    dws = [DevWeights(w) for w in ws_host]
+    w8s = [E4m3Weights(w, out_down) for w in ws_host]
+    x = dev_bf16(xb)
+    ws_b = h3.h3_workspace_size_e4m3(dl.dims, xb.shape[0], L.S)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+    h3.h3_stack_forward_e4m3(dl.dims, [w.c for w in dws], [w.c for w in w8s], dl.handle, tmod, x,
+                             xb.shape[0], ws, ws_b)
+    torch.cuda.synchronize()
+    assert h3.h3_layout_error(dl.handle) == h3.H3_OK
+    return host_f64(x)
+
+
+@pytest.mark.parametrize("out_down", [False, True])
+def test_e4m3_stack_small_amplified(out_down):
+    """Three 8-bit blocks through h3_stack_forward_e4m3 (fp32 residual stream)
+    against the oracle's 8-bit blocks in sequence, with the 8-bit block's budget."""
+    dims = SMALL
+    L = random_layout(256, 4, pad_runs=2, max_run=60)
+    ws_host = [amplified_weights(dims, 40 + i) for i in range(3)]
+    tm = (np.random.default_rng([4, 62]).standard_normal((L.n_t, 6, dims.hidden)) * 0.3
+          ).astype(np.float32)
+    xb = normal_bf16((1, L.S, dims.hidden), [4, 63], 1.0)
+    got = gpu_stack_e4m3(dims, L, ws_host, dev_f32(tm), xb, out_down)[0]
+    x0 = O.bf16_to_f64(xb[0])
+    ref, ref64 = _stack_refs(x0, ws_host, L, tm, dims, out_down)
+    pad = L.tags < 0
+    sp = Spread(ref, ref64, x0, ~pad)
+    assert_close_flips(got, ref, sp, what="e4m3 3-block stack x_out", storage_rounding=True)
+    assert_close(got[~pad] - x0[~pad], ref[~pad] - x0[~pad], what="e4m3 stack update",
+                 rel=REL_L2 + sp.upd, mabs=np.inf)
+    np.testing.assert_array_equal(got[pad], x0[pad])
+
+
+def test_e4m3_stack_full_width_two_blocks():
+    dims = FULL_DIMS
+    segs = [("text", 0, 300), ("video", (2, 16, 16), 0, 2), ("pad", 90), ("audio", 0, 598)]
+    L = make_layout(segs, seed=[19])
+    ws_host = [block_weights(dims, 9, i) for i in range(2)]
+    pw = prologue_weights(dims, 9)
+    xb = activations(dims, 9, L.S)
+    got = gpu_stack_e4m3(dims, L, ws_host, gpu_tmod(dims, L.timestep, pw), xb, True)[0]
+    x0 = O.bf16_to_f64(xb[0])
+    tm = O.timestep_modulation(L.timestep, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim, dims.hidden)
+    ref, ref64 = _stack_refs(x0, ws_host, L, tm, dims, True)
+    pad = L.tags < 0
+    sp = Spread(ref, ref64, x0, ~pad)
+    assert_close_flips(got, ref, sp, what="full-width e4m3 2-block stack x_out",
+                       storage_rounding=True)
+    assert_close(got[~pad] - x0[~pad], ref[~pad] - x0[~pad], what="full-width e4m3 stack update",
+                 rel=REL_L2 + sp.upd, mabs=np.inf)
+    np.testing.assert_array_equal(got[pad], x0[pad])
