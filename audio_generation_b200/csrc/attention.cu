@@ -33,6 +33,9 @@
 // valid, all padding or mixed, plus a valid-row bitmask. Key tiles that are
 // all padding are skipped; padding keys of mixed tiles are masked. Rows of
 // all-padding query tiles are written as zeros.
+// Output rows are placed through a RowMap (internal.cuh): the plain [B, S,
+// NH * 128] layout, or, for a rank of the sequence-parallel block, the receive
+// buffer of the rank that owns each row.
 #include "host_util.cuh"
 #include "internal.cuh"
 #include "sm100.cuh"

@@ -38,9 +38,13 @@
 //   EPI_SWIGLU W1 / W3 interleaved in 128-row blocks: g = SiLU(a) * b.
 //   EPI_STORE  plain bf16 store (the GEMM core on its own).
 //   EPI_F32    plain fp32 store (the prologue's split-operand GEMMs).
-// The QKV and SwiGLU epilogues also come in an e4m3 form (kind::f8f6f4 MMAs
-// over 128-element K stages of 8-bit codes), whose accumulator is multiplied
-// by the row's activation scale and the column's weight scale first.
+// The QKV, SwiGLU and gated-residual epilogues also come in an e4m3 form
+// (kind::f8f6f4 MMAs over 128-element K stages of 8-bit codes, BN = 256), whose
+// accumulator is multiplied by the row's activation scale and the column's
+// weight scale first.
+// EPI_QKV places each head's rows through a HeadMap (internal.cuh): the plain
+// block's [B, NH, S, 128] layout, or the receive buffers of the ranks of the
+// sequence-parallel block.
 #include "host_util.cuh"
 #include "internal.cuh"
 #include "sm100.cuh"
