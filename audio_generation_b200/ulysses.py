@@ -207,7 +207,10 @@ def symmetric_receive_buffers(dims, S: int, group=None):
             n *= d
         views.append(area[off:off + 2 * n].view(torch.bfloat16).view(*shp))
     ptrs = [int(p) for p in hdl.buffer_ptrs]
-    lists = [[p + off for p in ptrs] for off in offs]
+    # the area may sit at an offset inside the symmetric allocation: the same
+    # offset on every rank
+    base = area.data_ptr() - ptrs[hdl.rank]
+    lists = [[p + base + off for p in ptrs] for off in offs]
     return tuple(views), lists, hdl
 
 
