@@ -188,7 +188,7 @@ def receive_offsets(dims, S: int, world: int):
     return offs, at
 
 
-def symmetric_receive_buffers(dims, S: int, group=None):
+def symmetric_receive_buffers(dims, S: int, group=None, device=None):
     """Receive buffers in torch's symmetric memory, one area per rank at the
     same offsets: returns (this rank's q, k, v, o views, the peers of every
     rank's areas as lists of addresses (q, k, v, o), the handle)."""
@@ -197,8 +197,9 @@ def symmetric_receive_buffers(dims, S: int, group=None):
 
     world = dist.get_world_size(group)
     offs, size = receive_offsets(dims, S, world)
-    area = symm_mem.empty(size, dtype=torch.uint8, device=torch.device("cuda",
-                                                                       torch.cuda.current_device()))
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    area = symm_mem.empty(size, dtype=torch.uint8, device=device)
     hdl = symm_mem.rendezvous(area, group if group is not None else dist.group.WORLD)
     views = []
     for off, shp in zip(offs, receive_shapes(dims, S, world)):

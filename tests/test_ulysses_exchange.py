@@ -82,3 +82,37 @@ def test_fused_exchange_receive_areas_and_peer_table():
     assert [p.q[j] for j in range(P)] == lists[0] and [p.o[j] for j in range(P)] == lists[3]
     with pytest.raises(ValueError):
         h3.make_peers(0, *[[1] * 9] * 4)
+
+
+def test_symmetric_receive_buffers_address_arithmetic(monkeypatch):
+    """symmetric_receive_buffers on a fake symmetric-memory backend (CPU): the
+    views sit at the receive offsets of this rank's area, and every rank's peer
+    addresses are its buffer base plus the area's offset in the allocation plus
+    the view's offset."""
+    import types
+    import torch.distributed as dist
+    from audio_generation_b200 import ulysses as U
+    from workloads import Dims
+
+    dims = Dims(hidden=256, heads=8, head_dim=128, ffn=384, time_embed_dim=64, time_hidden=128)
+    S, P, rank = 64, 4, 2
+    pool = torch.zeros(1 << 20, dtype=torch.uint8)
+    lead = 512  # the area starts this far into the (fake) symmetric allocation
+
+    def empty(size, dtype=None, device=None):
+        return pool[lead:lead + size]
+
+    bases = [0x10000000 * (j + 1) for j in range(P)]
+    bases[rank] = pool.data_ptr()
+    hdl = types.SimpleNamespace(buffer_ptrs=bases, rank=rank)
+    fake = types.SimpleNamespace(empty=empty, rendezvous=lambda t, g: hdl)
+    monkeypatch.setitem(__import__("sys").modules, "torch.distributed._symmetric_memory", fake)
+    monkeypatch.setattr(dist, "get_world_size", lambda group=None: P)
+    monkeypatch.setattr(dist, "group", types.SimpleNamespace(WORLD="world"), raising=False)
+    views, lists, h = U.symmetric_receive_buffers(dims, S, group="g", device="cpu")
+    offs, size = U.receive_offsets(dims, S, P)
+    assert [tuple(v.shape) for v in views] == [tuple(s) for s in U.receive_shapes(dims, S, P)]
+    for v, off in zip(views, offs):
+        assert v.data_ptr() == pool.data_ptr() + lead + off
+    for lst, off in zip(lists, offs):
+        assert lst == [b + lead + off for b in bases]
