@@ -190,3 +190,28 @@ def test_noalloc_and_workspace_prologue_check_arguments_alike():
                                             None) == h3.H3_ERR_ARG
     assert L.h3_timestep_modulation_noalloc(ctypes.byref(d), 0, None, None, None, None, None,
                                             None) == h3.H3_OK
+
+
+def test_new_entry_points_reject_bad_arguments_on_the_host():
+    """The 8-bit steps and stack, and the sequence-parallel steps, return their
+    status before any device work for missing or inconsistent arguments."""
+    L = h3.lib()
+    d = h3.make_dims(FULL_DIMS)
+    fake = ctypes.c_void_p(256)  # never dereferenced: the checks fail first
+    # 8-bit stack: no operands, negative block count
+    w = h3.h3_block_weights()
+    assert L.h3_stack_forward_e4m3(ctypes.byref(d), ctypes.byref(w), None, 1, fake, fake, fake, 1,
+                                   fake, 1 << 30, None) == h3.H3_ERR_ARG
+    assert L.h3_stack_forward_e4m3(ctypes.byref(d), None, None, -1, fake, fake, fake, 1, fake, 0,
+                                   None) == h3.H3_ERR_ARG
+    # 8-bit residual steps without a layout
+    for fn in (L.h3_out_residual_e4m3, L.h3_ffn_down_residual_e4m3):
+        assert fn(ctypes.byref(d), None, 1, fake, fake, fake, fake, fake, fake, fake,
+                  None) == h3.H3_ERR_ARG
+    # sequence-parallel steps: no layout, no peer table
+    p = h3.make_peers(0, [256, 512], [256, 512], [256, 512], [256, 512])
+    assert L.h3_qkv_rope_to_heads(ctypes.byref(d), None, fake, fake, fake, fake, ctypes.byref(p),
+                                  None) == h3.H3_ERR_ARG
+    assert L.h3_attention_to_rows(ctypes.byref(d), None, fake, fake, fake, None,
+                                  None) == h3.H3_ERR_ARG
+    assert h3.H3_MAX_RANKS == 8
