@@ -160,11 +160,12 @@ def test_stack_config5_50_blocks_against_float64_golden(config5):
     Against the float64 golden: x_out and the stack's update x_out - x_in within
     rel-L2 1e-2; padding rows bit-identical. Against the oracle's bf16-storage
     golden of the same stack (bf16 at every operand the device stores in bf16,
-    the residual stream in fp32, as on the device): rel-L2 1e-2 and max-abs 5e-2
-    beyond the output's own bf16 rounding. The largest difference from the
-    float64 golden is held to 5e-2 plus the distance between the two goldens:
-    after 50 blocks the residual stream reaches |x| ~ 20, where the bf16 operand
-    roundings that any bf16 stack performs move the output by more than 5e-2."""
+    the residual stream in fp32, as on the device): rel-L2 1e-2. The largest
+    difference from either golden is held to 5e-2 plus the distance between the
+    two goldens (0.20 at |x| ~ 20; rel-L2 5.9e-3): after 50 blocks the bf16
+    operand roundings that any bf16 stack performs, an exactly rounded one
+    included, move the output by that much, and two stacks that round
+    differently part by as much."""
     g = _golden(GOLDEN5, config5)
     L, xb = config5["L"], config5["xb"]
     rows = g["rows"]
@@ -182,9 +183,10 @@ def test_stack_config5_50_blocks_against_float64_golden(config5):
     gb = _golden(GOLDEN5_BF16, config5)
     np.testing.assert_array_equal(gb["rows"], rows)
     ref16 = gb["x_out"].astype(np.float64)
-    assert_close(got, ref16, what="cfg5 50-block x_out vs bf16-storage golden",
-                 storage_rounding=True)
     spread = float(np.max(np.abs(ref16 - ref)))
+    assert spread > 5e-2  # the floor of a bf16 stack is above the per-block bound here
+    assert_close(got, ref16, what="cfg5 50-block x_out vs bf16-storage golden",
+                 mabs=5e-2 + spread)
     d = float(np.max(np.abs(got - ref)))
     assert d <= 5e-2 + spread, f"max-abs {d:.3e} vs float64 golden > 5e-2 + {spread:.3e}"
 
