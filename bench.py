@@ -538,11 +538,21 @@ def run_gpu(args, world, rank, local):
         # the 50-block stack over the padded 16384-row layout, two timed forwards
         del x_host, out_host, xd, ws
         torch.cuda.empty_cache()
-        st = stack_measure(2, 1)
+        st = stack_measure(2, 1, reduce_blocks=(3, 39))
         line["stack_config5"] = {k: st[k] for k in ("value", "unit", "ms_per_step", "tflops",
                                                     "frac_of_sustained_peak", "frac_of_burst_peak",
-                                                    "clocks", "steps", "warmup")}
+                                                    "clocks", "steps", "warmup", "token_reduced")}
         line["stack_config5"]["workload"] = st["config"]["workload"]
+        torch.cuda.empty_cache()
+        # the same stack with every GEMM on e4m3 operands, and the 8-bit block
+        s8 = stack_measure(2, 1, e4m3=True)
+        line["stack_config5_e4m3"] = {k: s8[k] for k in ("value", "unit", "ms_per_step", "tflops",
+                                                         "dtype", "clocks")}
+        torch.cuda.empty_cache()
+        b8 = e4m3_measure(10, 3, cfg)
+        line["block_e4m3"] = {k: b8[k] for k in ("value", "unit", "ms_per_step", "tflops", "dtype",
+                                                 "clocks", "qkv_w13_only")}
+        torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_baseline(cfg, args.ref_rows, 3)
     if rank == 0:
@@ -774,7 +784,7 @@ def stack_measure(steps, warmup, reduce_blocks=None, e4m3=False):
     return line
 
 
-def run_e4m3(args):
+def e4m3_measure(steps, warmup, cfg):
     """--e4m3: the block step of the workload with all four GEMMs (QKV, O,
     W1 || W3, W2) on e4m3 operands (h3_block_forward_e4m3; weights quantized once,
     before timing; o and g quantized per row inside the step), and the form with
@@ -787,7 +797,6 @@ def run_e4m3(args):
     torch.cuda.set_device(device)
     dims = FULL_DIMS
     d = h3.make_dims(dims)
-    cfg = args.workload
     L = config_layout(cfg)
     S, V = L.S, L.n_valid
     bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(
@@ -827,16 +836,16 @@ def run_e4m3(args):
         h3.h3_block_forward_e4m3(d, cw, ww, layout, tmod, x, 1, ws, ws_b, stream)
 
     # the form with QKV and W1 || W3 only, timed first
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step(w8_two)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step(w8_two)
     t1.record(stream)
     torch.cuda.synchronize(device)
-    ms_two = t0.elapsed_time(t1) / args.steps
-    for _ in range(args.warmup):
+    ms_two = t0.elapsed_time(t1) / steps
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize(device)
     gpu_id = torch.cuda.get_device_properties(device).uuid
@@ -845,19 +854,19 @@ def run_e4m3(args):
     with ClockSampler(gpu_id) as clk:
         time.sleep(0.3)
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize(device)
     if h3.h3_layout_error(layout) != h3.H3_OK:
         raise RuntimeError("device error word set during the e4m3 run")
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = e0.elapsed_time(e1) / steps
     tflops = block_flops(dims, V) / (ms * 1e-3) / 1e12
     peaks = load_peaks()
     line = {
         "metric": METRIC + " [e4m3 operands for QKV, O, W1||W3 and W2]",
         "value": S / (ms * 1e-3),
-        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": warmup, "ms_per_step": ms,
         "higher_is_better": True, "dtype": "e4m3 (QKV, O, W1||W3, W2) + bf16 (attention)",
         "data": "synthetic (seeded random-init weights and activations)",
         "config": {"workload": WORKLOADS[cfg], "S": S, "valid_rows": V},
@@ -866,9 +875,8 @@ def run_e4m3(args):
         "qkv_w13_only": {"ms_per_step": ms_two, "value": S / (ms_two * 1e-3),
                          "tflops": block_flops(dims, V) / (ms_two * 1e-3) / 1e12},
     }
-    print(json.dumps(line))
     layout.close()
-    return 0
+    return line
 
 
 FORWARD_WORKLOAD = ("full MiniMax-H3 transformer forward: fp32 patch projections (96 / 32 "
@@ -876,6 +884,11 @@ FORWARD_WORKLOAD = ("full MiniMax-H3 transformer forward: fp32 patch projections
                     "over the 16384-row padded layout (15872 valid rows, two timesteps), norm_out "
                     "and the fp32 video / audio heads")
 
+
+
+def run_e4m3(args):
+    print(json.dumps(e4m3_measure(args.steps, args.warmup, args.workload)))
+    return 0
 
 def run_forward(args):
     """--forward: one whole transformer forward (h3_forward) on one GPU, from
