@@ -890,6 +890,115 @@ def run_e4m3(args):
     print(json.dumps(e4m3_measure(args.steps, args.warmup, args.workload)))
     return 0
 
+
+def run_ulysses(args):
+    """--ulysses P: one rank's share of the sequence-parallel block on this GPU.
+    Rank 0 of P runs its row chunk's norm + QKV (storing each head's rows into
+    the owning rank's receive buffer), attention of its NH / P heads over every
+    row (storing each row's output into the owning rank's buffer) and its
+    chunk's O, norm and FFN. The receive buffers of all ranks live on this GPU,
+    so the exchange stores land in local memory: the figure is one rank's
+    compute, with the NVLink transfer time given beside it from the bytes each
+    rank sends and the measured 770 GB/s per direction. The plain block on the
+    same GPU is timed for comparison."""
+    import types
+    import torch
+    from audio_generation_b200 import h3
+    from audio_generation_b200.ulysses import UlyssesBlock
+
+    P = args.ulysses
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    dims = FULL_DIMS
+    d = h3.make_dims(dims)
+    cfg = args.workload
+    L = config_layout(cfg)
+    S, V = L.S, L.n_valid
+    if S % P or dims.heads % P or not 1 <= P <= 8:
+        raise SystemExit("--ulysses P needs S % P == 0, heads % P == 0 and P <= 8")
+    bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(
+        torch.bfloat16)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+    w = block_weights(dims, cfg, 0)
+    wd = types.SimpleNamespace(**{k: bits(getattr(w, k)) for k in ("w_qkv", "q_norm", "k_norm",
+                                                                  "w_o", "w13", "w2")})
+    wd.ada_table = f32(w.ada_table)
+    pw = prologue_weights(dims, cfg)
+    tws_b = h3.h3_timestep_workspace_size(d, L.n_t)
+    tws = torch.empty(tws_b, dtype=torch.uint8, device=device)
+    tmod = torch.empty((L.n_t, 6, dims.hidden), dtype=torch.float32, device=device)
+    h3.h3_timestep_modulation(d, L.n_t, f32(L.timestep), f32(pw.w_t1), f32(pw.w_t2),
+                              f32(pw.w_proj), tmod, tws, tws_b)
+    del tws
+    xb = activations(dims, cfg, S, 1)
+    ranks = [UlyssesBlock(dims, L, r, P, device) for r in range(P)]
+    Sr, NHl, D, H = S // P, dims.heads // P, dims.head_dim, dims.hidden
+    peers = [h3.make_peers(r, *[[ranks[j].recv[i] for j in range(P)] for i in range(4)])
+             for r in range(P)]
+    xs = [bits(np.ascontiguousarray(xb[:, r * Sr:(r + 1) * Sr])) for r in range(P)]
+    for r, rk in enumerate(ranks):  # every rank's q, k, v in place before rank 0's attention
+        rk.pre_attention_to_heads(wd, tmod, xs[r], peers[r])
+    x0 = xs[0].clone()
+    stream = torch.cuda.current_stream(device)
+    r0 = ranks[0]
+
+    def rank0_step():
+        xs[0].copy_(x0)
+        r0.pre_attention_to_heads(wd, tmod, xs[0], peers[0])
+        r0.attention_to_rows(peers[0])
+        r0.post_attention(wd, tmod, r0.recv[3][None], xs[0])
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / args.steps
+
+    ms_rank = timed(rank0_step)
+    for rk in ranks:
+        if h3.h3_layout_error(rk.full) != h3.H3_OK or h3.h3_layout_error(rk.chunk) != h3.H3_OK:
+            raise RuntimeError("device error word set during the sequence-parallel run")
+        rk.close()
+    del ranks, peers, xs, r0
+    torch.cuda.empty_cache()
+    # the plain block on the same GPU
+    layout = h3.h3_layout_prepare(d, S, L.n_t, f32(L.pos), i32(L.tags), i32(L.t_idx),
+                                  i32(L.video_idx), i32(L.audio_idx), i32(L.text_idx))
+    cw = h3.make_block_weights(wd.w_qkv, wd.q_norm, wd.k_norm, wd.w_o, wd.w13, wd.w2,
+                               wd.ada_table)
+    x = bits(xb)
+    ws_b = h3.h3_workspace_size(d, 1, S)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=device)
+    ms_block = timed(lambda: h3.h3_block_forward(d, cw, layout, tmod, x, 1, ws, ws_b, stream))
+    layout.close()
+    # bytes one rank sends: q, k, v of its rows for the other ranks' heads, and
+    # the attention output of the other ranks' rows for its heads
+    out_bytes = 3 * Sr * (dims.heads - NHl) * D * 2 + (S - Sr) * NHl * D * 2
+    line = {
+        "metric": f"one rank's compute per block step, sequence-parallel over {P} ranks "
+                  "(bf16, measured on 1xB200, exchange stores to local memory)",
+        "value": ms_rank, "unit": "ms", "higher_is_better": False, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights and activations)",
+        "config": {"workload": WORKLOADS[cfg], "S": S, "valid_rows": V, "ranks": P,
+                   "rows_per_rank": Sr, "heads_per_rank": NHl},
+        "single_gpu_block_ms": ms_block,
+        "per_rank_share_of_block": ms_rank / ms_block,
+        "exchange_bytes_sent_per_rank": out_bytes,
+        "exchange_ms_at_770_GBps": out_bytes / 770e9 * 1e3,
+        "note": "a P-GPU step is at least the per-rank compute; the exchange is stored by the "
+                "producing kernels and overlaps them on NVLink, not measured here",
+    }
+    print(json.dumps(line))
+    return 0
+
 def run_forward(args):
     """--forward: one whole transformer forward (h3_forward) on one GPU, from
     latent rows to velocities. Prints one JSON line: forward time, valid rows/s
@@ -1020,6 +1129,8 @@ def main(argv=None):
                     help="skip the 50-block stack measurement added to the block line")
     ap.add_argument("--no-masked", action="store_true",
                     help="skip the masked-attention measurement on the padded layout")
+    ap.add_argument("--ulysses", type=int, default=0,
+                    help="time one rank's share of the sequence-parallel block over this many ranks")
     ap.add_argument("--reduced", action="store_true",
                     help="with --stack: also time the token-reduced stack")
     ap.add_argument("--stack", action="store_true",
@@ -1036,6 +1147,8 @@ def main(argv=None):
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.ulysses:
+        return run_ulysses(args)
     if args.stack:
         return run_stack(args)
     if args.forward:
