@@ -61,3 +61,40 @@ def test_sample_rows_cover_padding_edges_and_mixed_tiles():
     assert np.any((rows >= 896) & (rows < 960)) and np.any((rows >= 1088) & (rows < 1152))
     L2 = random_layout(500, 3, pad_runs=3)
     assert sample_rows(L2).size >= 64
+
+
+def test_head_parallel_pieces_keep_the_bf16_storage_emulation():
+    """The --emulate golden: the pieces pass the emulation through (P rounded
+    per row, as the whole attention does), and the block in its bf16-storage,
+    fp32-stream reading is unchanged by the piecewise attention."""
+    g = np.random.default_rng(12)
+    q = g.standard_normal((40, 3, 128))
+    k = g.standard_normal((33, 3, 128))
+    v = g.standard_normal((33, 3, 128))
+    dk = g.random(33) < 0.2
+    dq = g.random(40) < 0.2
+    dk[0], dk[1] = False, True
+    ref = O.attention(q, dq, k, v, dk, emulate=True)
+    got = head_parallel_attention(3, q_chunk=16)(q, dq, k, v, dk, emulate=True)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+    assert not np.allclose(ref, O.attention(q, dq, k, v, dk), rtol=1e-6)  # emulation is on
+
+    from workloads import TINY_DIMS, activations, block_weights, prologue_weights
+    dims = TINY_DIMS
+    L = config_layout(1)
+    w = block_weights(dims, 1, 0)
+    pw = prologue_weights(dims, 1)
+    x = O.bf16_to_f64(activations(dims, 1, L.S))
+    tm = O.timestep_modulation(L.timestep, pw.w_t1, pw.w_t2, pw.w_proj, dims.freq_dim,
+                               dims.hidden)
+    ref = O.block_forward(x, w, L, tm, dims, emulate=True, stream_f32=True)
+    base = O.attention
+    try:
+        O.attention = head_parallel_attention(4)
+        got = O.block_forward(x, w, L, tm, dims, emulate=True, stream_f32=True)
+    finally:
+        O.attention = base
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+    # the fp32 stream: x1 and the output are fp32 values, not bf16 ones
+    assert np.array_equal(got, got.astype(np.float32).astype(np.float64))
+    assert not np.array_equal(got, O.round_bf16(got))
